@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Benchmark of one Ulysses attention layer step on B200.
+
+A step is the whole hot path over one batch: seq->head permute (Q, K, V),
+causal GQA flash attention forward, head->seq permute (O), seq->head permute
+(dO), attention backward, head->seq permute (dQ, dK, dV). Default workload:
+packed varlen, N = 65536 tokens, P = 4 virtual ranks, H = 32, H_kv = 8, d = 128
+("Ulysses layer tokens/s & attn TFLOP/s at 64K tokens; permute HBM GB/s").
+
+Prints one JSON line (rank 0). Multi-GPU (torchrun): every rank runs its own
+independent layer (replicas; the path has no cross-GPU step on one GPU's
+emulated ranks), value = total tokens of all ranks / max-over-ranks time.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(MEASURED_PEAKS) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def flops(w, cu):
+    pairs = workloads.causal_pairs(w.N, cu)
+    return 4.0 * w.d * w.H * pairs, 10.0 * w.d * w.H * pairs, pairs
+
+
+def permute_bytes(w):
+    """Algorithmic bytes of each permute launch (read + write once)."""
+    q = w.N * w.H * w.d * 2
+    kv = w.N * w.H_kv * w.d * 2
+    return {"qkv_s2h": 2 * (q + 2 * kv), "o_h2s": 2 * q, "do_s2h": 2 * q, "dqkv_h2s": 2 * (q + 2 * kv)}
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_oracle_sample(w, inp, budget_s=20.0):
+    """Time the fp64 oracle on a bounded sample of the workload and extrapolate
+    the layer time linearly in (i, j) pairs x heads. Sample: forward + backward
+    of the first document (or the first 2048 tokens), one kv head group
+    (H/H_kv query heads), plus the three permutes of that slice."""
+    import oracle
+    cu = inp["cu_seqlens"]
+    L = int(cu[1]) if cu is not None else min(w.N, 2048)
+    L = min(L, 4096)
+    group = w.H // w.H_kv
+    widen = oracle.widen_bf16
+    q = widen(inp["q"][:L, :group])
+    k = widen(inp["k"][:L, :1])
+    v = widen(inp["v"][:L, :1])
+    do = widen(inp["do"][:L, :group]) if "do" in inp else None
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.attention_forward(q, k, v)
+        if do is not None:
+            oracle.attention_backward(q, k, v, do)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s / 2 or reps >= 50:
+            break
+    t_attn = (time.perf_counter() - t0) / reps
+    sample_pairs = L * (L + 1) // 2 * group
+    full_pairs = workloads.causal_pairs(w.N, cu) * w.H
+    t_attn_full = t_attn * full_pairs / sample_pairs
+    # permutes: time the oracle's seq->head on a token slice and scale by bytes
+    sl = min(w.N, 8192)
+    xs = workloads.seq_shards(inp["q"][:sl], w.P)
+    t1 = time.perf_counter()
+    preps = 0
+    while time.perf_counter() - t1 < min(2.0, budget_s / 4):
+        oracle.head_to_seq(oracle.seq_to_head(xs))
+        preps += 1
+    t_perm = (time.perf_counter() - t1) / preps / 2       # one permute of the Q slice
+    q_bytes = sl * w.H * w.d * 2
+    perm_bytes_step = sum(permute_bytes(w).values()) / 2  # tensor bytes moved (each read+write counted once)
+    t_perm_full = t_perm * perm_bytes_step / q_bytes
+    t_layer = t_attn_full + t_perm_full
+    cores = len(os.sched_getaffinity(0))
+    return {
+        "value": w.N / t_layer, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+        "sample": (f"fp64 numpy oracle fwd{'+bwd' if do is not None else ''} on the first {L} tokens x "
+                   f"{group} query heads (1 kv head), {reps} reps, {t_attn:.3f} s each, plus seq<->head "
+                   f"permutes of {sl} tokens; extrapolated linearly by (i,j)-pairs x heads and by bytes"),
+        "t_layer_s": t_layer, "t_sample_s": t_attn,
+    }
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inp = workloads.generate(w, N=min(w.N, 16384) if w.varlen is None else None)
+    budget = 10.0
+    vals = []
+    t_all = time.perf_counter()
+    for s in range(args.warmup + args.steps):
+        cb = cpu_oracle_sample(w, inp, budget_s=budget)
+        if s >= args.warmup:
+            vals.append(cb)
+    v = statistics.median([c["value"] for c in vals])
+    cb = vals[-1]
+    line = {
+        "impl": "reference", "metric": "Ulysses layer tokens/s (fwd+bwd)" if w.backward else "Ulysses layer tokens/s (fwd)",
+        "value": v, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * w.N / v, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "N": w.N, "P": w.P, "H": w.H, "H_kv": w.H_kv, "d": w.d},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cb["cores"], "kind": "oracle",
+                         "sample": cb["sample"]},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": time.perf_counter() - t_all,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="varlen64k", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    w = workloads.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    import ulysses_sequence_parallelism_b200 as U
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    inp = workloads.generate(w, seed=0)
+    cu_np = inp["cu_seqlens"]
+    cu = None if cu_np is None else torch.tensor(cu_np, dtype=torch.int32, device=dev)
+    P, H, H_kv, d, N = w.P, w.H, w.H_kv, w.d, w.N
+    layer = U.UlyssesLayer(N, P, H, H_kv, d, device=dev, cu_seqlens=cu, backward=w.backward,
+                           rank_sequential=w.rank_sequential)
+
+    def shards(x):
+        n = N // P
+        return [torch.from_numpy(x[p * n:(p + 1) * n].view(np.int16)).view(torch.bfloat16).to(dev) for p in range(P)]
+
+    q, k, v = shards(inp["q"]), shards(inp["k"]), shards(inp["v"])
+    do = shards(inp["do"]) if w.backward else None
+    o = [torch.empty_like(x) for x in q]
+    if w.backward:
+        dq = [torch.empty_like(x) for x in q]
+        dk = [torch.empty_like(x) for x in k]
+        dv = [torch.empty_like(x) for x in v]
+    stream = torch.cuda.current_stream()
+
+    f_fwd, f_bwd, pairs = flops(w, cu_np)
+    pb = permute_bytes(w)
+    stages = ["qkv_s2h", "attn_fwd", "o_h2s"] + (["do_s2h", "attn_bwd", "dqkv_h2s"] if w.backward else [])
+
+    def step(ev=None):
+        """One layer step; ev: list of len(stages)+1 events to record between stages."""
+        L = layer
+        if ev: ev[0].record(stream)
+        U.ulysses_a2a_seq_to_head(q, k, v, L.q_h, L.k_h, L.v_h, N, P, H, H_kv, d, cu)
+        if ev: ev[1].record(stream)
+        U.ulysses_attn_fwd(L.q_h, L.k_h, L.v_h, L.o_h, L.lse, N, P, H, H_kv, d, cu)
+        if ev: ev[2].record(stream)
+        U.ulysses_a2a_head_to_seq(L.o_h, None, None, o, None, None, N, P, H, H_kv, d, cu)
+        if ev: ev[3].record(stream)
+        if w.backward:
+            U.ulysses_a2a_seq_to_head(do, None, None, L.do_h, None, None, N, P, H, H_kv, d, cu)
+            if ev: ev[4].record(stream)
+            U.ulysses_attn_bwd(L.q_h, L.k_h, L.v_h, L.o_h, L.lse, L.do_h, L.dq_h, L.dk_h, L.dv_h, N, P, H, H_kv, d,
+                               L.workspace, cu)
+            if ev: ev[5].record(stream)
+            U.ulysses_a2a_head_to_seq(L.dq_h, L.dk_h, L.dv_h, dq, dk, dv, N, P, H, H_kv, d, cu)
+            if ev: ev[6].record(stream)
+
+    if w.rank_sequential:
+        raise SystemExit("bench.py times all-rank workloads; the million-token workload is a parity case")
+
+    launches_per_step = 1 + 1 + 1 + ((1 + 3 + 1) if w.backward else 0)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    code, word = U.ulysses_get_device_status()
+    if code != 0:
+        raise SystemExit(f"device status {code} word {word:#x} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_begin.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    total_ms = t_begin.elapsed_time(t_end)
+    stage_ms = {st: [] for st in stages}
+    for s in range(args.steps):
+        for i, st in enumerate(stages):
+            stage_ms[st].append(evs[s][i].elapsed_time(evs[s][i + 1]))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * N / (ms_per_step / 1e3)
+
+    med = {st: statistics.median(v_) for st, v_ in stage_ms.items()}
+    mean = {st: sum(v_) / len(v_) for st, v_ in stage_ms.items()}
+    peaks, peak_src = load_peaks()
+    fwd_tflops = f_fwd / (mean["attn_fwd"] / 1e3) / 1e12
+    perm_gbs = {st: pb[st] / (mean[st] / 1e3) / 1e9 for st in pb if st in mean}
+    detail = {"attn_fwd_tflops": fwd_tflops, "permute_gbs": perm_gbs,
+              "stage_ms_mean": mean, "stage_ms_median": med, "pairs": pairs, "attn_fwd_flops": f_fwd}
+    if w.backward:
+        detail["attn_bwd_tflops"] = f_bwd / (mean["attn_bwd"] / 1e3) / 1e12
+        detail["attn_bwd_flops"] = f_bwd
+    # dominant kernel by measured time
+    dom = max(mean, key=mean.get)
+    tensor_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    if dom in ("attn_fwd", "attn_bwd"):
+        achieved = (f_fwd if dom == "attn_fwd" else f_bwd) / (mean[dom] / 1e3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": achieved / tensor_peak, "traffic": None,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)"}
+    else:
+        achieved = pb[dom] / (mean[dom] / 1e3) / 1e9
+        hp = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hp, "unit": "GB/s",
+                "frac": achieved / hp, "traffic": None, "peak_source": f"{peak_src} hbm_gbs"}
+
+    # ---------------------------------------------------------------- end to end through the public API
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+        n = N // P
+        hq = [pin(inp["q"][p * n:(p + 1) * n]) for p in range(P)]
+        hk = [pin(inp["k"][p * n:(p + 1) * n]) for p in range(P)]
+        hv = [pin(inp["v"][p * n:(p + 1) * n]) for p in range(P)]
+        hdo = [pin(inp["do"][p * n:(p + 1) * n]) for p in range(P)] if w.backward else []
+        outs_h = [torch.empty_like(x).pin_memory() for x in hq]
+        if w.backward:
+            outs_h += [torch.empty_like(x).pin_memory() for x in hq + hk + hv]
+        dev_in = q + k + v + (do if w.backward else [])
+        host_in = hq + hk + hv + hdo
+        dev_out = o + ((dq + dk + dv) if w.backward else [])
+        h2d = sum(x.numel() * 2 for x in host_in)
+        d2h = sum(x.numel() * 2 for x in outs_h)
+
+        def e2e_step():
+            for hsrc, dd in zip(host_in, dev_in):
+                dd.copy_(hsrc, non_blocking=True)
+            layer.forward(q, k, v, o)
+            if w.backward:
+                layer.backward(do, dq, dk, dv)
+            for dsrc, hh in zip(dev_out, outs_h):
+                hh.copy_(dsrc, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / args.steps
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * N / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_oracle_sample(w, inp, budget_s=20.0)
+        cpu = {k_: cb[k_] for k_ in ("value", "unit", "cores", "kind", "sample")}
+
+    if rank == 0:
+        line = {
+            "metric": "Ulysses layer tokens/s (fwd+bwd)" if w.backward else "Ulysses layer tokens/s (fwd)",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "N": N, "P": P, "H": H, "H_kv": H_kv, "d": d,
+                       "docs": None if cu_np is None else int(len(cu_np) - 1),
+                       "pass": "fwd+bwd" if w.backward else "fwd",
+                       "l2": "inputs larger than L2 (per-tensor working sets 0.27-1.3 GB > 126 MB); no flush",
+                       "parallelism": f"{P} virtual ranks per GPU; {world} independent replica(s)"},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk, "detail": detail,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

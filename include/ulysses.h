@@ -1,0 +1,158 @@
+/*
+ * ulysses.h -- C ABI of the single-GPU Ulysses sequence-parallel attention layer
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The layer (theaicatchup.com, "How Does Ulysses Sequence Parallelism Actually
+ * Work?"; radardeia.com, "Arquitetura Técnica"): every rank holds a contiguous
+ * chunk of N/P tokens; an all-to-all turns that into all N positions for H/P
+ * heads; each rank runs full-sequence causal attention on its heads (heads are
+ * independent); the inverse all-to-all returns the output to sequence sharding.
+ * Here the P ranks are P disjoint device buffers on one GPU, so each
+ * all-to-all is an on-device permute.
+ *
+ * Layouts (all row-major, bf16 unless stated):
+ *   sequence shard, rank p : [N/P, Hx, d]   token t = p*N/P + s
+ *   head shard, rank p     : [N, Hx/P, d]   local head j = global head p*Hx/P + j
+ *   LSE, rank p            : float32 [H/P, N] (natural log of the scaled scores' sum)
+ *   Hx = H for Q, O, dO, dQ;  Hx = H_kv for K, V, dK, dV.
+ *   Query head h reads key/value head h / (H/H_kv).
+ *
+ * Conventions for every entry point:
+ *   - Rank buffers are passed as HOST arrays of P DEVICE pointers, indexed by
+ *     rank. Entries of ranks outside [rank_lo, rank_hi) are not read and may
+ *     be NULL. The caller owns all device memory (including workspace); the
+ *     library never allocates or frees device memory.
+ *   - Every device pointer must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream) and do
+ *     not synchronise, except ulysses_get_device_status().
+ *   - Arguments are validated before any launch. On ULY_ERR_INVALID_ARG or
+ *     ULY_ERR_UNSUPPORTED nothing is launched and no memory is touched. A
+ *     launch failure returns ULY_ERR_CUDA. Nothing aborts or traps.
+ *   - Supported shapes: 1 <= P <= ULY_MAX_RANKS; N % P == 0; H % P == 0;
+ *     H_kv % P == 0 (the pages' "num_heads >= sp_size", strengthened so that
+ *     heads split evenly -- contenidos2-1ml.pages.dev, "¿Qué cambia en la
+ *     práctica...?"); H % H_kv == 0; d in {64, 128}; N/P*H*d < 2^31.
+ *   - cu_seqlens: DEVICE int32 array [num_seqs+1], cu_seqlens[0] = 0,
+ *     non-decreasing, cu_seqlens[num_seqs] = N (packed variable-length
+ *     documents, block-diagonal causal mask). NULL = one causal sequence.
+ *     The kernels clamp what they read, so malformed contents give wrong
+ *     numbers but never an out-of-bounds access.
+ */
+#ifndef ULYSSES_B200_H
+#define ULYSSES_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ULY_MAX_RANKS 16
+
+#if defined(__GNUC__)
+#define ULY_API __attribute__((visibility("default")))
+#else
+#define ULY_API
+#endif
+
+typedef enum {
+  ULY_OK = 0,
+  ULY_ERR_INVALID_ARG = 1,   /* bad pointer, size, range or alignment */
+  ULY_ERR_UNSUPPORTED = 2,   /* valid but not implemented (d, P, causal=0, ...) */
+  ULY_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+  ULY_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up (see get_device_status) */
+} uly_status;
+
+/* All-to-all #1, sequence sharding -> head sharding (theaicatchup.com, "How Does
+ * Ulysses...": "every GPU ends up with all positions, but only a slice of heads").
+ *   dst[q][t, j, :] = src[t / (N/P)][t % (N/P), q*Hx/P + j, :]
+ * Up to three tensors move in one launch: slot 0 has H heads (Q, or dO in the
+ * backward), slots 1 and 2 have H_kv heads (K, V). A NULL slot-1/2 array skips
+ * that tensor. Only destination ranks q in [rank_lo, rank_hi) are written
+ * (0..P for all); every source rank is read. cu_seqlens/num_seqs are accepted
+ * for symmetry and ignored (the permute is a pure index map; documents may
+ * straddle shards). Bit-exact copy. */
+ULY_API uly_status ulysses_a2a_seq_to_head(
+    const void* const* x0_seq, const void* const* x1_seq, const void* const* x2_seq,
+    void* const* x0_head, void* const* x1_head, void* const* x2_head,
+    int64_t N, int P, int H, int H_kv, int d,
+    const int32_t* cu_seqlens, int num_seqs,
+    int rank_lo, int rank_hi, cudaStream_t stream);
+
+/* All-to-all #2, head sharding -> sequence sharding: the exact inverse of
+ * ulysses_a2a_seq_to_head ("Reverse the shuffle", theaicatchup.com, ibid.;
+ * "Reconstrução Contextual", radardeia.com).
+ *   dst[p][s, q*Hx/P + j, :] = src[q][p*N/P + s, j, :]
+ * Slot 0: H heads (O; dQ in the backward); slots 1, 2: H_kv heads (dK, dV).
+ * Only SOURCE ranks q in [rank_lo, rank_hi) are read, i.e. only their head
+ * columns of every destination shard are written. Bit-exact copy. */
+ULY_API uly_status ulysses_a2a_head_to_seq(
+    const void* const* x0_head, const void* const* x1_head, const void* const* x2_head,
+    void* const* x0_seq, void* const* x1_seq, void* const* x2_seq,
+    int64_t N, int P, int H, int H_kv, int d,
+    const int32_t* cu_seqlens, int num_seqs,
+    int rank_lo, int rank_hi, cudaStream_t stream);
+
+/* Causal (optionally packed-varlen) grouped-query flash attention forward on the
+ * head shards of ranks [rank_lo, rank_hi) ("Compute attention locally",
+ * theaicatchup.com, ibid.; heads are independent, ibid., quoting DeepSpeed-Ulysses):
+ *   s_ij = softmax_scale * q_i.k_j  for j <= i in the same document,
+ *   o_i = sum_j softmax_j(s_i) v_j  (bf16, round to nearest even),
+ *   lse_i = ln sum_j exp(s_ij)      (float32, layout [H/P, N]).
+ * Inputs q_head (H/P heads), k_head/v_head (H_kv/P heads) per rank; outputs
+ * o_head and lse_head per rank. softmax_scale <= 0 selects 1/sqrt(d).
+ * causal must be 1 (ULY_ERR_UNSUPPORTED otherwise). max_seqlen is a hint
+ * (longest document; <= 0 = unknown). fp32 accumulation and softmax. */
+ULY_API uly_status ulysses_attn_fwd(
+    const void* const* q_head, const void* const* k_head, const void* const* v_head,
+    void* const* o_head, float* const* lse_head,
+    int64_t N, int P, int H, int H_kv, int d,
+    const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
+    float softmax_scale, int causal,
+    int rank_lo, int rank_hi, cudaStream_t stream);
+
+/* Bytes of device workspace ulysses_attn_bwd needs for these sizes (fp32 dQ
+ * accumulator and the per-row D_i = dO_i . O_i), for all P ranks. */
+ULY_API size_t ulysses_attn_bwd_workspace_size(int64_t N, int P, int H, int H_kv, int d);
+
+/* Attention backward on the head shards of ranks [rank_lo, rank_hi). The pages
+ * train through the layer but do not write its backward; this is the gradient
+ * of the forward above (softmax-attention calculus):
+ *   P_ij = exp(s_ij - lse_i), D_i = dO_i . O_i,
+ *   dV_j = sum_i P_ij dO_i,   dS_ij = P_ij (dO_i.v_j - D_i),
+ *   dQ_i = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i,
+ * with dK/dV summed over the H/H_kv query heads of each group. Inputs: q, k, v,
+ * o, do_head (head shards, as in the forward) and lse_head from the forward.
+ * Outputs dq_head (H/P heads), dk_head, dv_head (H_kv/P heads), bf16.
+ * workspace: caller-owned device memory of at least
+ * ulysses_attn_bwd_workspace_size() bytes, 256-byte aligned; its contents on
+ * entry do not matter. */
+ULY_API uly_status ulysses_attn_bwd(
+    const void* const* q_head, const void* const* k_head, const void* const* v_head,
+    const void* const* o_head, const float* const* lse_head, const void* const* do_head,
+    void* const* dq_head, void* const* dk_head, void* const* dv_head,
+    int64_t N, int P, int H, int H_kv, int d,
+    const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
+    float softmax_scale,
+    void* workspace, size_t workspace_bytes,
+    int rank_lo, int rank_hi, cudaStream_t stream);
+
+/* Static text for a status code. */
+ULY_API const char* ulysses_status_string(uly_status s);
+
+/* Reads and clears the library's device-side error word on the current device
+ * (set by a bounded wait that gave up, or by a kernel's own bounds check).
+ * Synchronises `stream`. Returns ULY_OK, ULY_ERR_TIMEOUT or ULY_ERR_CUDA;
+ * *detail (may be NULL) receives the raw word (0 = clean). */
+ULY_API uly_status ulysses_get_device_status(cudaStream_t stream, uint32_t* detail);
+
+/* Test hook: caps every bounded device-side wait at `iters` polls (0 restores
+ * the default). Lets a host test make a wait run out without faulting the GPU. */
+ULY_API void ulysses_set_wait_limit(uint32_t iters);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ULYSSES_B200_H */

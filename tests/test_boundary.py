@@ -1,0 +1,104 @@
+"""C-ABI library: it loads, exports every symbol include/ulysses.h declares, and
+its host-side validation rejects bad arguments before any launch. No compute
+call is made here (these run without a GPU: validation returns before the
+CUDA runtime is touched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ulysses.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from ulysses_sequence_parallelism_b200 import build
+    build.build()
+    from ulysses_sequence_parallelism_b200 import _lib
+    return _lib.lib()
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"ULY_API\s+[\w\s\*]+?\b(ulysses_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_four_layer_entry_points():
+    syms = declared_symbols()
+    for s in ("ulysses_a2a_seq_to_head", "ulysses_a2a_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_bwd"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    from ulysses_sequence_parallelism_b200 import _lib
+    for s in declared_symbols():
+        assert hasattr(L, s), s
+    assert set(declared_symbols()) <= set(_lib.exported_symbols()) | set(declared_symbols())
+    assert set(_lib.exported_symbols()) <= set(declared_symbols())
+
+
+def test_status_strings(L):
+    assert L.ulysses_status_string(0) == b"ok"
+    assert L.ulysses_status_string(1) == b"invalid argument"
+    assert L.ulysses_status_string(4) == b"bounded device wait timed out"
+
+
+def _arr(vals):
+    a = (ctypes.c_void_p * len(vals))(*vals)
+    return ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p))
+
+
+GOOD = 0x10000   # a 16-byte aligned fake device address: never dereferenced (validation fails first)
+
+
+def _fwd(L, N=256, P=2, H=8, H_kv=8, d=64, ptr=GOOD, causal=1, lo=0, hi=None, cu=None, ns=0, lse_ptr=GOOD):
+    p = _arr([ptr] * P)
+    lp = _arr([lse_ptr] * P)
+    return L.ulysses_attn_fwd(p, p, p, p, lp, N, P, H, H_kv, d, cu, ns, 0, 0.0, causal, lo,
+                              P if hi is None else hi, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(P=0), 1), (dict(N=0), 1), (dict(N=255), 1),             # N % P
+    (dict(H=8, H_kv=3, P=1), 1),                                   # H % H_kv
+    (dict(P=16, N=256, H=8, H_kv=8), 1),                           # H < P  (num_heads >= sp_size)
+    (dict(H=8, H_kv=2, P=4), 1),                                   # H_kv % P: kv heads must split too
+    (dict(P=17, N=17 * 16, H=17, H_kv=17), 2),                     # more ranks than supported
+    (dict(d=96), 2), (dict(d=256), 2),                             # head dims not built
+    (dict(causal=0), 2),                                           # non-causal not built
+    (dict(lo=1, hi=1), 1), (dict(lo=-1), 1), (dict(hi=3), 1),      # rank range
+    (dict(ptr=0), 1), (dict(ptr=GOOD + 8), 1), (dict(lse_ptr=GOOD + 4), 1),   # null / misaligned
+    (dict(cu=ctypes.c_void_p(GOOD), ns=0), 1),                     # cu_seqlens with no documents
+])
+def test_attn_fwd_validation(L, kw, code):
+    assert _fwd(L, **kw) == code
+
+
+def test_a2a_validation(L):
+    P = 2
+    p = _arr([GOOD] * P)
+    bad = _arr([GOOD, GOOD + 2])
+    # slot 1/2 must be given on both sides or neither
+    assert L.ulysses_a2a_seq_to_head(p, p, None, p, None, None, 256, P, 8, 8, 64, None, 0, 0, P, None) == 1
+    assert L.ulysses_a2a_seq_to_head(bad, None, None, p, None, None, 256, P, 8, 8, 64, None, 0, 0, P, None) == 1
+    assert L.ulysses_a2a_head_to_seq(p, None, None, bad, None, None, 256, P, 8, 8, 64, None, 0, 0, P, None) == 1
+    assert L.ulysses_a2a_seq_to_head(p, None, None, p, None, None, 256, P, 8, 8, 48, None, 0, 0, P, None) == 2
+    # a NULL head-side buffer of a rank inside the range is rejected
+    half = _arr([GOOD, 0])
+    assert L.ulysses_a2a_seq_to_head(p, None, None, half, None, None, 256, P, 8, 8, 64, None, 0, 0, P, None) == 1
+
+
+def test_bwd_validation_and_workspace_size(L):
+    ws = L.ulysses_attn_bwd_workspace_size(8192, 4, 32, 8, 128)
+    assert ws >= 4 * 8192 * 8 * 128 * 4 + 4 * 8192 * 8 * 4
+    assert L.ulysses_attn_bwd_workspace_size(8192, 3, 32, 8, 128) == 0     # invalid shape -> 0
+    P = 2
+    p = _arr([GOOD] * P)
+    # workspace too small / misaligned
+    assert L.ulysses_attn_bwd(p, p, p, p, p, p, p, p, p, 256, P, 8, 8, 64, None, 0, 0, 0.0,
+                              ctypes.c_void_p(GOOD), 16, 0, P, None) == 1
+    need = L.ulysses_attn_bwd_workspace_size(256, P, 8, 8, 64)
+    assert L.ulysses_attn_bwd(p, p, p, p, p, p, p, p, p, 256, P, 8, 8, 64, None, 0, 0, 0.0,
+                              ctypes.c_void_p(GOOD + 16), need, 0, P, None) == 1

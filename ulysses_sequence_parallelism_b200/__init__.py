@@ -1,0 +1,13 @@
+"""Ulysses sequence-parallel attention layer for NVIDIA B200 (sm_100a).
+
+The C ABI (``include/ulysses.h``) lives in ``libulysses_b200.so``, built
+in-tree by ``build.py``; this package is a thin ctypes binding over it.
+"""
+from ._lib import UlyssesError, lib, LIB_PATH, exported_symbols
+from .api import (ulysses_a2a_seq_to_head, ulysses_a2a_head_to_seq, ulysses_attn_fwd, ulysses_attn_bwd,
+                  ulysses_attn_bwd_workspace_size, ulysses_get_device_status, ulysses_set_wait_limit,
+                  UlyssesLayer)
+
+__all__ = ["UlyssesError", "lib", "LIB_PATH", "exported_symbols", "ulysses_a2a_seq_to_head",
+           "ulysses_a2a_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_bwd", "ulysses_attn_bwd_workspace_size",
+           "ulysses_get_device_status", "ulysses_set_wait_limit", "UlyssesLayer"]

@@ -1,0 +1,180 @@
+"""Thin Python binding over the C ABI (argument marshalling only).
+
+Each function takes per-rank lists of CUDA tensors, checks dtype/device/
+contiguity, passes raw device pointers plus the current CUDA stream to the
+library, and raises ``UlyssesError`` on a non-zero status. Every step of the
+layer runs in the library's kernels; PyTorch provides device memory and
+streams. Shapes follow ``include/ulysses.h``:
+
+  sequence shard of rank p : [N/P, Hx, d] bf16
+  head shard of rank p     : [N, Hx/P, d] bf16
+  LSE of rank p            : [H/P, N] float32
+"""
+import ctypes
+from typing import List, Optional, Sequence
+
+import torch
+
+from ._lib import lib, check, UlyssesError, MAX_RANKS
+
+__all__ = [
+    "ulysses_a2a_seq_to_head", "ulysses_a2a_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_bwd",
+    "ulysses_attn_bwd_workspace_size", "ulysses_get_device_status", "ulysses_set_wait_limit", "UlyssesLayer",
+]
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptrs(ts: Optional[Sequence[Optional[torch.Tensor]]], P: int, dtype=torch.bfloat16):
+    if ts is None:
+        return None
+    if len(ts) != P:
+        raise ValueError(f"expected {P} rank tensors, got {len(ts)}")
+    arr = (ctypes.c_void_p * P)()
+    for r, t in enumerate(ts):
+        if t is None:
+            arr[r] = None
+            continue
+        if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+            raise ValueError(f"rank {r}: need a contiguous CUDA {dtype} tensor, got {t.dtype} on {t.device}")
+        arr[r] = t.data_ptr()
+    return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+
+
+def _cu(cu_seqlens: Optional[torch.Tensor]):
+    if cu_seqlens is None:
+        return None, 0
+    if not cu_seqlens.is_cuda or cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be a CUDA int32 tensor")
+    return ctypes.c_void_p(cu_seqlens.data_ptr()), cu_seqlens.numel() - 1
+
+
+def ulysses_a2a_seq_to_head(x0_seq, x1_seq, x2_seq, x0_head, x1_head, x2_head, N, P, H, H_kv, d,
+                            cu_seqlens=None, rank_lo=0, rank_hi=None, stream=None):
+    cu, ns = _cu(cu_seqlens)
+    code = lib().ulysses_a2a_seq_to_head(
+        _ptrs(x0_seq, P), _ptrs(x1_seq, P), _ptrs(x2_seq, P), _ptrs(x0_head, P), _ptrs(x1_head, P),
+        _ptrs(x2_head, P), N, P, H, H_kv, d, cu, ns, rank_lo, P if rank_hi is None else rank_hi, _stream(stream))
+    check("ulysses_a2a_seq_to_head", code)
+
+
+def ulysses_a2a_head_to_seq(x0_head, x1_head, x2_head, x0_seq, x1_seq, x2_seq, N, P, H, H_kv, d,
+                            cu_seqlens=None, rank_lo=0, rank_hi=None, stream=None):
+    cu, ns = _cu(cu_seqlens)
+    code = lib().ulysses_a2a_head_to_seq(
+        _ptrs(x0_head, P), _ptrs(x1_head, P), _ptrs(x2_head, P), _ptrs(x0_seq, P), _ptrs(x1_seq, P),
+        _ptrs(x2_seq, P), N, P, H, H_kv, d, cu, ns, rank_lo, P if rank_hi is None else rank_hi, _stream(stream))
+    check("ulysses_a2a_head_to_seq", code)
+
+
+def ulysses_attn_fwd(q_head, k_head, v_head, o_head, lse_head, N, P, H, H_kv, d, cu_seqlens=None,
+                     max_seqlen=0, softmax_scale=0.0, causal=1, rank_lo=0, rank_hi=None, stream=None):
+    cu, ns = _cu(cu_seqlens)
+    code = lib().ulysses_attn_fwd(
+        _ptrs(q_head, P), _ptrs(k_head, P), _ptrs(v_head, P), _ptrs(o_head, P), _ptrs(lse_head, P, torch.float32),
+        N, P, H, H_kv, d, cu, ns, max_seqlen, float(softmax_scale), causal, rank_lo,
+        P if rank_hi is None else rank_hi, _stream(stream))
+    check("ulysses_attn_fwd", code)
+
+
+def ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d) -> int:
+    return int(lib().ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d))
+
+
+def ulysses_attn_bwd(q_head, k_head, v_head, o_head, lse_head, do_head, dq_head, dk_head, dv_head, N, P, H,
+                     H_kv, d, workspace: torch.Tensor, cu_seqlens=None, max_seqlen=0, softmax_scale=0.0,
+                     rank_lo=0, rank_hi=None, stream=None):
+    cu, ns = _cu(cu_seqlens)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    code = lib().ulysses_attn_bwd(
+        _ptrs(q_head, P), _ptrs(k_head, P), _ptrs(v_head, P), _ptrs(o_head, P), _ptrs(lse_head, P, torch.float32),
+        _ptrs(do_head, P), _ptrs(dq_head, P), _ptrs(dk_head, P), _ptrs(dv_head, P), N, P, H, H_kv, d, cu, ns,
+        max_seqlen, float(softmax_scale), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), rank_lo, P if rank_hi is None else rank_hi, _stream(stream))
+    check("ulysses_attn_bwd", code)
+
+
+def ulysses_get_device_status(stream=None):
+    """Synchronises the stream, reads and clears the device error word.
+    Returns (status_code, raw_word)."""
+    w = ctypes.c_uint32(0)
+    code = lib().ulysses_get_device_status(_stream(stream), ctypes.byref(w))
+    return code, w.value
+
+
+def ulysses_set_wait_limit(iters: int):
+    lib().ulysses_set_wait_limit(int(iters))
+
+
+class UlyssesLayer:
+    """One Ulysses attention layer over P virtual ranks of one GPU.
+
+    Holds the head-sharded buffers (and the backward workspace) so repeated
+    steps allocate nothing. ``forward`` runs seq->head (Q, K, V in one launch),
+    attention forward, head->seq (O); ``backward`` runs seq->head (dO),
+    attention backward, head->seq (dQ, dK, dV in one launch)."""
+
+    def __init__(self, N: int, P: int, H: int, H_kv: int, d: int, device="cuda", cu_seqlens=None,
+                 max_seqlen: int = 0, softmax_scale: float = 0.0, backward: bool = True,
+                 rank_sequential: bool = False):
+        if P > MAX_RANKS:
+            raise ValueError(f"P <= {MAX_RANKS}")
+        self.N, self.P, self.H, self.H_kv, self.d = N, P, H, H_kv, d
+        self.cu = cu_seqlens
+        self.max_seqlen = max_seqlen
+        self.scale = softmax_scale
+        self.rank_sequential = rank_sequential
+        bf, f32 = torch.bfloat16, torch.float32
+        nb = 1 if rank_sequential else P      # rank-sequential: one rank's head buffers, reused
+        mk = lambda hx: [torch.empty(N, hx // P, d, dtype=bf, device=device) for _ in range(nb)]
+        self.q_h, self.k_h, self.v_h, self.o_h = mk(H), mk(H_kv), mk(H_kv), mk(H)
+        self.lse = [torch.empty(H // P, N, dtype=f32, device=device) for _ in range(nb)]
+        self.backward_enabled = backward and not rank_sequential
+        if self.backward_enabled:
+            self.do_h, self.dq_h, self.dk_h, self.dv_h = mk(H), mk(H), mk(H_kv), mk(H_kv)
+            ws = ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d)
+            self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
+
+    def _rank_bufs(self, bufs, r):
+        lst = [None] * self.P
+        lst[r] = bufs[0]
+        return lst
+
+    def forward(self, q_seq: List[torch.Tensor], k_seq, v_seq, o_seq: Optional[List[torch.Tensor]] = None):
+        N, P, H, H_kv, d = self.N, self.P, self.H, self.H_kv, self.d
+        if o_seq is None:
+            o_seq = [torch.empty_like(x) for x in q_seq]
+        if not self.rank_sequential:
+            ulysses_a2a_seq_to_head(q_seq, k_seq, v_seq, self.q_h, self.k_h, self.v_h, N, P, H, H_kv, d, self.cu)
+            ulysses_attn_fwd(self.q_h, self.k_h, self.v_h, self.o_h, self.lse, N, P, H, H_kv, d, self.cu,
+                             self.max_seqlen, self.scale)
+            ulysses_a2a_head_to_seq(self.o_h, None, None, o_seq, None, None, N, P, H, H_kv, d, self.cu)
+        else:
+            for r in range(P):
+                rb = lambda b: self._rank_bufs(b, r)
+                ulysses_a2a_seq_to_head(q_seq, k_seq, v_seq, rb(self.q_h), rb(self.k_h), rb(self.v_h), N, P, H,
+                                        H_kv, d, self.cu, rank_lo=r, rank_hi=r + 1)
+                ulysses_attn_fwd(rb(self.q_h), rb(self.k_h), rb(self.v_h), rb(self.o_h), rb(self.lse), N, P, H,
+                                 H_kv, d, self.cu, self.max_seqlen, self.scale, rank_lo=r, rank_hi=r + 1)
+                ulysses_a2a_head_to_seq(rb(self.o_h), None, None, o_seq, None, None, N, P, H, H_kv, d, self.cu,
+                                        rank_lo=r, rank_hi=r + 1)
+        return o_seq
+
+    def backward(self, do_seq: List[torch.Tensor], dq_seq=None, dk_seq=None, dv_seq=None):
+        if not self.backward_enabled:
+            raise RuntimeError("layer built without backward buffers")
+        N, P, H, H_kv, d = self.N, self.P, self.H, self.H_kv, self.d
+        if dq_seq is None:
+            dq_seq = [torch.empty(N // P, H, d, dtype=torch.bfloat16, device=do_seq[0].device) for _ in range(P)]
+            dk_seq = [torch.empty(N // P, H_kv, d, dtype=torch.bfloat16, device=do_seq[0].device) for _ in range(P)]
+            dv_seq = [torch.empty(N // P, H_kv, d, dtype=torch.bfloat16, device=do_seq[0].device) for _ in range(P)]
+        ulysses_a2a_seq_to_head(do_seq, None, None, self.do_h, None, None, N, P, H, H_kv, d, self.cu)
+        ulysses_attn_bwd(self.q_h, self.k_h, self.v_h, self.o_h, self.lse, self.do_h, self.dq_h, self.dk_h,
+                         self.dv_h, N, P, H, H_kv, d, self.workspace, self.cu, self.max_seqlen, self.scale)
+        ulysses_a2a_head_to_seq(self.dq_h, self.dk_h, self.dv_h, dq_seq, dk_seq, dv_seq, N, P, H, H_kv, d, self.cu)
+        return dq_seq, dk_seq, dv_seq

@@ -1,0 +1,164 @@
+// C-ABI entry points: argument validation, then the kernel launchers.
+// Nothing here allocates, frees or synchronises device memory except
+// ulysses_get_device_status / ulysses_set_wait_limit, which touch the
+// library's own device words.
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ulysses.h"
+
+namespace {
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+uly_status check_shape(int64_t N, int P, int H, int H_kv, int d, int rank_lo, int rank_hi) {
+  if (P < 1 || N <= 0 || H <= 0 || H_kv <= 0) return ULY_ERR_INVALID_ARG;
+  if (P > ULY_MAX_RANKS) return ULY_ERR_UNSUPPORTED;
+  if (N % P != 0 || H % P != 0 || H_kv % P != 0 || H % H_kv != 0) return ULY_ERR_INVALID_ARG;
+  if (rank_lo < 0 || rank_hi > P || rank_lo >= rank_hi) return ULY_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ULY_ERR_UNSUPPORTED;
+  if (N > INT32_MAX || (N / P) * static_cast<int64_t>(H) * d >= (int64_t(1) << 31) ||
+      N * static_cast<int64_t>(H / P) * d >= (int64_t(1) << 31))
+    return ULY_ERR_UNSUPPORTED;
+  return ULY_OK;
+}
+
+// Every entry of ranks [lo, hi) must be a 16-byte aligned non-null pointer.
+bool ranks_ok(const void* const* arr, int lo, int hi) {
+  if (arr == nullptr) return false;
+  for (int r = lo; r < hi; ++r)
+    if (!aligned16(arr[r])) return false;
+  return true;
+}
+
+uly_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ULY_OK : ULY_ERR_CUDA; }
+
+uly_status check_cu(const int32_t* cu, int num_seqs, int64_t N) {
+  if (cu == nullptr) return ULY_OK;
+  if (num_seqs < 1 || num_seqs > N) return ULY_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu) & 3u) != 0) return ULY_ERR_INVALID_ARG;
+  return ULY_OK;
+}
+
+uly_status a2a(bool seq_to_head, const void* const* s0, const void* const* s1, const void* const* s2,
+               void* const* d0, void* const* d1, void* const* d2, int64_t N, int P, int H, int H_kv, int d,
+               const int32_t* cu, int num_seqs, int rank_lo, int rank_hi, cudaStream_t stream) {
+  uly_status st = check_shape(N, P, H, H_kv, d, rank_lo, rank_hi);
+  if (st != ULY_OK) return st;
+  if (check_cu(cu, num_seqs, N) != ULY_OK) return ULY_ERR_INVALID_ARG;
+  if (s0 == nullptr || d0 == nullptr) return ULY_ERR_INVALID_ARG;
+  if ((s1 == nullptr) != (d1 == nullptr) || (s2 == nullptr) != (d2 == nullptr)) return ULY_ERR_INVALID_ARG;
+  if (H * (d / 8) > uly::permute_max_row_vecs()) return ULY_ERR_UNSUPPORTED;
+  // Sequence side: every rank. Head side: ranks in range.
+  const void* const* src[3] = {s0, s1, s2};
+  void* const* dst[3] = {d0, d1, d2};
+  for (int s = 0; s < 3; ++s) {
+    if (src[s] == nullptr) continue;
+    const int slo = seq_to_head ? 0 : rank_lo, shi = seq_to_head ? P : rank_hi;
+    const int dlo = seq_to_head ? rank_lo : 0, dhi = seq_to_head ? rank_hi : P;
+    if (!ranks_ok(src[s], slo, shi) || !ranks_ok(reinterpret_cast<const void* const*>(dst[s]), dlo, dhi))
+      return ULY_ERR_INVALID_ARG;
+  }
+  const int hx[3] = {H, H_kv, H_kv};
+  return from_cuda(uly::launch_permute(seq_to_head, src, dst, hx, N, P, d, rank_lo, rank_hi, stream));
+}
+
+float resolve_scale(float softmax_scale, int d) {
+  return (softmax_scale > 0.f && isfinite(softmax_scale)) ? softmax_scale : 1.0f / sqrtf(static_cast<float>(d));
+}
+
+}  // namespace
+
+extern "C" {
+
+uly_status ulysses_a2a_seq_to_head(const void* const* x0_seq, const void* const* x1_seq, const void* const* x2_seq,
+                                   void* const* x0_head, void* const* x1_head, void* const* x2_head, int64_t N,
+                                   int P, int H, int H_kv, int d, const int32_t* cu_seqlens, int num_seqs,
+                                   int rank_lo, int rank_hi, cudaStream_t stream) {
+  return a2a(true, x0_seq, x1_seq, x2_seq, x0_head, x1_head, x2_head, N, P, H, H_kv, d, cu_seqlens, num_seqs,
+             rank_lo, rank_hi, stream);
+}
+
+uly_status ulysses_a2a_head_to_seq(const void* const* x0_head, const void* const* x1_head,
+                                   const void* const* x2_head, void* const* x0_seq, void* const* x1_seq,
+                                   void* const* x2_seq, int64_t N, int P, int H, int H_kv, int d,
+                                   const int32_t* cu_seqlens, int num_seqs, int rank_lo, int rank_hi,
+                                   cudaStream_t stream) {
+  return a2a(false, x0_head, x1_head, x2_head, x0_seq, x1_seq, x2_seq, N, P, H, H_kv, d, cu_seqlens, num_seqs,
+             rank_lo, rank_hi, stream);
+}
+
+uly_status ulysses_attn_fwd(const void* const* q_head, const void* const* k_head, const void* const* v_head,
+                            void* const* o_head, float* const* lse_head, int64_t N, int P, int H, int H_kv, int d,
+                            const int32_t* cu_seqlens, int num_seqs, int max_seqlen, float softmax_scale,
+                            int causal, int rank_lo, int rank_hi, cudaStream_t stream) {
+  (void)max_seqlen;
+  uly_status st = check_shape(N, P, H, H_kv, d, rank_lo, rank_hi);
+  if (st != ULY_OK) return st;
+  if (causal != 1) return ULY_ERR_UNSUPPORTED;
+  if (check_cu(cu_seqlens, num_seqs, N) != ULY_OK) return ULY_ERR_INVALID_ARG;
+  if (!ranks_ok(q_head, rank_lo, rank_hi) || !ranks_ok(k_head, rank_lo, rank_hi) ||
+      !ranks_ok(v_head, rank_lo, rank_hi) || !ranks_ok(reinterpret_cast<const void* const*>(o_head), rank_lo, rank_hi) ||
+      !ranks_ok(reinterpret_cast<const void* const*>(lse_head), rank_lo, rank_hi))
+    return ULY_ERR_INVALID_ARG;
+  uly::AttnShape s{static_cast<int>(N), P, H / P, H_kv / P, d, cu_seqlens, cu_seqlens ? num_seqs : 1,
+                   resolve_scale(softmax_scale, d), rank_lo, rank_hi};
+  return from_cuda(uly::launch_attn_fwd(s, q_head, k_head, v_head, o_head, lse_head, stream));
+}
+
+size_t ulysses_attn_bwd_workspace_size(int64_t N, int P, int H, int H_kv, int d) {
+  if (check_shape(N, P, H, H_kv, d, 0, P > 0 ? P : 1) != ULY_OK) return 0;
+  return uly::attn_bwd_workspace_bytes(N, P, H / P, d);
+}
+
+uly_status ulysses_attn_bwd(const void* const* q_head, const void* const* k_head, const void* const* v_head,
+                            const void* const* o_head, const float* const* lse_head, const void* const* do_head,
+                            void* const* dq_head, void* const* dk_head, void* const* dv_head, int64_t N, int P,
+                            int H, int H_kv, int d, const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
+                            float softmax_scale, void* workspace, size_t workspace_bytes, int rank_lo,
+                            int rank_hi, cudaStream_t stream) {
+  (void)max_seqlen;
+  uly_status st = check_shape(N, P, H, H_kv, d, rank_lo, rank_hi);
+  if (st != ULY_OK) return st;
+  if (check_cu(cu_seqlens, num_seqs, N) != ULY_OK) return ULY_ERR_INVALID_ARG;
+  auto cv = [](void* const* p) { return reinterpret_cast<const void* const*>(p); };
+  if (!ranks_ok(q_head, rank_lo, rank_hi) || !ranks_ok(k_head, rank_lo, rank_hi) ||
+      !ranks_ok(v_head, rank_lo, rank_hi) || !ranks_ok(o_head, rank_lo, rank_hi) ||
+      !ranks_ok(reinterpret_cast<const void* const*>(lse_head), rank_lo, rank_hi) ||
+      !ranks_ok(do_head, rank_lo, rank_hi) || !ranks_ok(cv(dq_head), rank_lo, rank_hi) ||
+      !ranks_ok(cv(dk_head), rank_lo, rank_hi) || !ranks_ok(cv(dv_head), rank_lo, rank_hi))
+    return ULY_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ULY_ERR_INVALID_ARG;
+  if (workspace_bytes < uly::attn_bwd_workspace_bytes(N, P, H / P, d)) return ULY_ERR_INVALID_ARG;
+  uly::AttnShape s{static_cast<int>(N), P, H / P, H_kv / P, d, cu_seqlens, cu_seqlens ? num_seqs : 1,
+                   resolve_scale(softmax_scale, d), rank_lo, rank_hi};
+  return from_cuda(uly::launch_attn_bwd(s, q_head, k_head, v_head, o_head, lse_head, do_head, dq_head, dk_head,
+                                        dv_head, workspace, stream));
+}
+
+const char* ulysses_status_string(uly_status s) {
+  switch (s) {
+    case ULY_OK: return "ok";
+    case ULY_ERR_INVALID_ARG: return "invalid argument";
+    case ULY_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case ULY_ERR_CUDA: return "CUDA runtime error";
+    case ULY_ERR_TIMEOUT: return "bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+uly_status ulysses_get_device_status(cudaStream_t stream, uint32_t* detail) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return ULY_ERR_CUDA;
+  uint32_t w = 0;
+  if (cudaMemcpyFromSymbol(&w, uly::g_error_word, sizeof(w)) != cudaSuccess) return ULY_ERR_CUDA;
+  const uint32_t zero = 0;
+  if (w != 0 && cudaMemcpyToSymbol(uly::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return ULY_ERR_CUDA;
+  if (detail) *detail = w;
+  return w == 0 ? ULY_OK : ULY_ERR_TIMEOUT;
+}
+
+void ulysses_set_wait_limit(uint32_t iters) { cudaMemcpyToSymbol(uly::g_wait_limit, &iters, sizeof(iters)); }
+
+}  // extern "C"

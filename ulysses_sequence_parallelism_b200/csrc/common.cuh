@@ -1,0 +1,117 @@
+// Shared device helpers for the Ulysses B200 kernels (sm_100a).
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#define ULY_DEV __device__ __forceinline__
+
+namespace uly {
+
+constexpr int kMaxRanks = 16;
+
+// Per-rank pointer tables, passed by value as kernel parameters.
+struct RankPtrs {
+  const void* p[kMaxRanks];
+};
+struct RankPtrsMut {
+  void* p[kMaxRanks];
+};
+struct RankPtrsF {
+  float* p[kMaxRanks];
+};
+struct RankPtrsFC {
+  const float* p[kMaxRanks];
+};
+
+// Library-wide device error word (bounded waits that gave up, bounds checks).
+// Bit layout: [31:24] kernel id, [23:0] site-specific detail. The library is
+// one translation unit, so these are defined here.
+__device__ uint32_t g_error_word = 0;
+// Poll cap for every bounded device-side wait (0 = the kernel's default).
+__device__ uint32_t g_wait_limit = 0;
+
+enum ErrKernel : uint32_t { kErrFwd = 1u, kErrBwd = 2u, kErrPermute = 3u };
+
+ULY_DEV void report_error(uint32_t kernel, uint32_t detail) {
+  atomicCAS(&g_error_word, 0u, (kernel << 24) | (detail & 0xFFFFFFu));
+}
+
+// ----------------------------------------------------------------- small math
+ULY_DEV float ex2_approx(float x) {
+  float y;
+  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+ULY_DEV uint32_t pack_bf16x2(float lo, float hi) {
+  // cvt.rn.bf16x2.f32 d, a, b puts a in the upper half and b in the lower half.
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// First token of the document containing row i (cu_seqlens may be null).
+// Clamped into [0, i] whatever the array holds.
+ULY_DEV int doc_start_of(const int32_t* __restrict__ cu, int num_seqs, int i) {
+  if (cu == nullptr) return 0;
+  int lo = 0, hi = num_seqs;  // find the last m with cu[m] <= i
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= i) lo = mid; else hi = mid - 1;
+  }
+  int s = __ldg(cu + lo);
+  return s < 0 ? 0 : (s > i ? i : s);
+}
+
+// One past the last token of the document containing row i, clamped into [i+1, N].
+ULY_DEV int doc_end_of(const int32_t* __restrict__ cu, int num_seqs, int i, int N) {
+  if (cu == nullptr) return N;
+  int lo = 0, hi = num_seqs;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= i) lo = mid; else hi = mid - 1;
+  }
+  int e = (lo + 1 <= num_seqs) ? __ldg(cu + lo + 1) : N;
+  return e <= i ? i + 1 : (e > N ? N : e);
+}
+
+// ----------------------------------------------------------------- mma.sync helpers
+ULY_DEV uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+ULY_DEV void cp_async_16(uint32_t smem, const void* gmem, bool pred) {
+  int sz = pred ? 16 : 0;  // src-size 0 zero-fills the 16 bytes
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem), "l"(gmem), "r"(sz));
+}
+ULY_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+ULY_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
+
+ULY_DEV void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+ULY_DEV void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32 accumulate.
+ULY_DEV void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a [rows][D] bf16 tile
+// whose 16-byte chunks are XOR-swizzled by (row & 7) (conflict-free ldmatrix).
+template <int D>
+ULY_DEV uint32_t swz(int row, int chunk) {
+  return static_cast<uint32_t>(row * (D * 2) + ((chunk ^ (row & 7)) << 4));
+}
+
+}  // namespace uly

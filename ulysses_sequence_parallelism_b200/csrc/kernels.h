@@ -1,0 +1,33 @@
+// Host-side launchers shared between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace uly {
+
+struct AttnShape {
+  int N;          // tokens (all ranks)
+  int P;          // virtual ranks
+  int Hl;         // query heads per rank (H/P)
+  int Hkvl;       // key/value heads per rank (H_kv/P)
+  int d;          // head dim
+  const int32_t* cu_seqlens;   // device, or null
+  int num_seqs;
+  float scale;    // softmax scale (already resolved; > 0)
+  int rank_lo, rank_hi;
+};
+
+int permute_max_row_vecs();
+cudaError_t launch_permute(bool seq_to_head, const void* const* src[3], void* const* dst[3], const int hx[3],
+                           int64_t N, int P, int d, int rank_lo, int rank_hi, cudaStream_t stream);
+
+cudaError_t launch_attn_fwd(const AttnShape& s, const void* const* q, const void* const* k,
+                            const void* const* v, void* const* o, float* const* lse, cudaStream_t stream);
+
+size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d);
+cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void* const* k,
+                            const void* const* v, const void* const* o, const float* const* lse,
+                            const void* const* dO, void* const* dq, void* const* dk, void* const* dv,
+                            void* workspace, cudaStream_t stream);
+
+}  // namespace uly

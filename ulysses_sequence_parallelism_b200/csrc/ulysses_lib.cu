@@ -1,0 +1,7 @@
+// Single translation unit for the whole library: the kernels share the
+// library's device-side error word and wait cap without relocatable device code.
+#include <string.h>
+#include "permute.cu"
+#include "attn_fwd_mma.cu"
+#include "attn_bwd_mma.cu"
+#include "api.cu"
