@@ -3,7 +3,7 @@ and compare against the fp64 oracle with the stated tolerances."""
 import numpy as np
 import torch
 
-# Parity bar for bf16 attention outputs and gradients (O, dQ, dK, dV):
+# Parity bar for bf16 attention outputs and gradients (O, dQ, dK, dV); see assert_close:
 MAX_ABS = 2e-2
 REL_RMS = 1e-2
 # LSE is float32 end to end; its error comes from the fp32 online softmax and the
@@ -30,6 +30,14 @@ def shards_to_dev(bits: np.ndarray, P: int):
     return [to_dev(bits[p * n:(p + 1) * n]) for p in range(P)]
 
 
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half the bf16 spacing at |x| (8 significant bits): the rounding error an
+    exact result already carries once stored as bf16 with round-to-nearest-even."""
+    ax = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, np.exp2(e - 8), 0.0)
+
+
 def err_stats(gpu: np.ndarray, ref: np.ndarray):
     e = gpu - ref
     ma = float(np.max(np.abs(e))) if e.size else 0.0
@@ -39,8 +47,21 @@ def err_stats(gpu: np.ndarray, ref: np.ndarray):
 
 
 def assert_close(name, gpu, ref, max_abs=MAX_ABS, rel_rms=REL_RMS):
-    ma, rr = err_stats(np.asarray(gpu, np.float64), np.asarray(ref, np.float64))
-    assert ma <= max_abs and rr <= rel_rms, f"{name}: max_abs {ma:.3e} (<= {max_abs}), rel_rms {rr:.3e} (<= {rel_rms})"
+    """Parity bar for bf16 results: relative RMS error <= rel_rms, and max
+    absolute error <= max_abs beyond the bf16 output's own half-ulp rounding
+    (an exact result stored in bf16 is already up to 2^-6 off at |x| in [4, 8),
+    2^-5 at [8, 16); the bar applies to the error the arithmetic adds)."""
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    ma, rr = err_stats(gpu, ref)
+    excess = np.abs(gpu - ref) - bf16_half_ulp(ref)
+    mx = float(np.max(excess)) if excess.size else 0.0
+    if not (mx <= max_abs and rr <= rel_rms):
+        i = np.unravel_index(int(np.argmax(excess)), excess.shape)
+        big = int(np.sum(np.abs(ref) >= 4.0))
+        raise AssertionError(
+            f"{name}: max_abs {ma:.3e}, beyond half-ulp {mx:.3e} (<= {max_abs}), rel_rms {rr:.3e} (<= {rel_rms}); "
+            f"worst at {i}: gpu {gpu[i]:.6f} ref {ref[i]:.6f}; {big} elements with |ref| >= 4")
     return ma, rr
 
 

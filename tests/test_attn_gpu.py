@@ -83,11 +83,15 @@ def test_layer_matches_oracle(N, P, H, H_kv, d, cu):
 
 
 def test_softmax_scale_argument():
+    """An explicit softmax_scale (0.09, not the default 1/sqrt(64) = 0.125) is
+    honoured by forward and backward."""
     N, P, H, H_kv, d = 192, 2, 4, 2, 64
     q, k, v, do = _draw(N, H, H_kv, d, seed=7)
-    gpu = run_gpu_layer(q, k, v, do, P, None, scale=0.3)
-    ref = oracle_layer(q, k, v, do, P, None, scale=0.3)
+    gpu = run_gpu_layer(q, k, v, do, P, None, scale=0.09)
+    ref = oracle_layer(q, k, v, do, P, None, scale=0.09)
     check(gpu, ref)
+    wrong = oracle_layer(q, k, v, do, P, None, scale=None)
+    assert np.max(np.abs(gpu["o"] - wrong["o"])) > 1e-2   # the default scale would not match
 
 
 def test_large_logits_stay_finite_and_exact():

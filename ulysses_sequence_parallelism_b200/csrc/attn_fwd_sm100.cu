@@ -1,0 +1,434 @@
+// Causal GQA (packed-varlen) flash-attention forward for sm_100a: tcgen05 MMA
+// with TMEM accumulators, TMA-fed shared-memory tiles, warp-specialised.
+//
+// Computes, per rank in range, per local query head h, per row i:
+//   s_ij = scale * q_i.k_j  (j <= i, same document),  o_i = softmax_j(s_i) V,
+//   lse_i = ln sum_j exp(s_ij)
+// ("Compute attention locally" on every rank's head slice over all positions,
+// heads being independent -- theaicatchup.com, "How Does Ulysses Sequence
+// Parallelism Actually Work?").
+//
+// One CTA owns two 128-row query tiles of one head (256 rows) and streams the
+// 128-key K/V blocks they need through a 4-stage shared-memory ring:
+//   warp 8      : TMA producer (Q tiles once, then K_j, V_j alternately)
+//   warp 9      : MMA issuer: S_t = Q_t K_j^T (SS, K-major both), then
+//                 O_t += P_t V_j (A = P from TMEM, B = V MN-major)
+//   warps 0-3/4-7: softmax of tile 0 / tile 1, one thread per row: reads its
+//                 S row from TMEM, online softmax in the log2 domain with fp32
+//                 statistics, writes P (bf16) back over S, rescales its O row
+//                 in TMEM only when its running max grew by more than 2^8
+//                 (the result is exact either way: O and l share the max),
+//                 and finally normalises O and stores O and LSE.
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
+// Every wait on an mbarrier is bounded; a wait that runs out records an error
+// in the library's device error word and the CTA drains and exits.
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace uly {
+namespace fwd_sm100 {
+
+using namespace sm100;
+
+constexpr int BM = 128;        // query rows per tile (two tiles per CTA)
+constexpr int BN = 128;        // keys per K/V block
+constexpr int NSTAGE = 4;      // K/V ring stages (K and V blocks alternate)
+constexpr int kThreads = 320;  // 8 softmax warps + TMA warp + MMA warp
+constexpr int kTmaWarp = 8, kMmaWarp = 9;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O when the max grows by > 2^8
+
+struct FwdArgs {
+  CUtensorMap tq[kMaxRanks];
+  CUtensorMap tk[kMaxRanks];
+  CUtensorMap tv[kMaxRanks];
+  RankPtrsMut o;
+  RankPtrsF lse;
+  const int32_t* cu;
+  int num_seqs;
+  int N, Hl, Hkvl, group;
+  float scale_log2;
+  int rank_lo;
+  int num_m_blocks;   // blocks of 2*BM rows
+};
+
+template <int D>
+struct Layout {
+  static constexpr uint32_t kQTile = BM * D * 2;       // bytes of one Q tile
+  static constexpr uint32_t kKV = BN * D * 2;          // bytes of one K or V block
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kRing = kQ + 2 * kQTile;
+  static constexpr uint32_t kBars = kRing + NSTAGE * kKV;
+  // barriers: q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], mma_done
+  static constexpr int kNumBars = 2 + 2 * NSTAGE + 2 + 2 + 2 + 1;
+  static constexpr uint32_t kTmemSlot = kBars + kNumBars * 8;
+  static constexpr uint32_t kBytes = kTmemSlot + 16;
+  static constexpr uint32_t kAlloc = kBytes + 1024;    // slack for 1024-byte alignment
+};
+
+ULY_DEV float u2f(uint32_t x) { return __uint_as_float(x); }
+ULY_DEV float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __grid_constant__ FwdArgs a) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  const uint32_t sQ = sbase + L::kQ, sRing = sbase + L::kRing, bars = sbase + L::kBars;
+  auto q_full = [&](int t) { return bars + 8u * t; };
+  auto kv_full = [&](int s) { return bars + 8u * (2 + s); };
+  auto kv_empty = [&](int s) { return bars + 8u * (2 + NSTAGE + s); };
+  auto s_full = [&](int t) { return bars + 8u * (2 + 2 * NSTAGE + t); };
+  auto p_full = [&](int t) { return bars + 8u * (4 + 2 * NSTAGE + t); };
+  auto pv_done = [&](int t) { return bars + 8u * (6 + 2 * NSTAGE + t); };
+  const uint32_t mma_done = bars + 8u * (8 + 2 * NSTAGE);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kTmemSlot);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x % a.Hl;
+  const int r = a.rank_lo + blockIdx.x / a.Hl;
+  const int g = h / a.group;
+  const int N = a.N;
+  const int m0 = (a.num_m_blocks - 1 - static_cast<int>(blockIdx.y)) * (2 * BM);   // longest first
+
+  // Per-tile row and key-block ranges (identical in every thread).
+  bool active[2];
+  int jb_begin[2], jb_end[2], first_row[2], last_row[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    first_row[t] = m0 + t * BM;
+    last_row[t] = min(first_row[t] + BM, N) - 1;
+    active[t] = first_row[t] < N;
+    if (active[t]) {
+      jb_begin[t] = doc_start_of(a.cu, a.num_seqs, first_row[t]) / BN;
+      jb_end[t] = last_row[t] / BN + 1;
+    } else {
+      jb_begin[t] = jb_end[t] = 0;
+    }
+  }
+  const int jb_lo = jb_begin[0];
+  const int jb_hi = active[1] ? max(jb_end[0], jb_end[1]) : jb_end[0];
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::kNumBars; ++i) mbar_init(bars + 8u * i, 1);
+    mbar_init(p_full(0), 128);
+    mbar_init(p_full(1), 128);
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(sbase + L::kTmemSlot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS[2] = {tmem, tmem + 128};
+  const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const CUtensorMap* mq = &a.tq[r];
+      const CUtensorMap* mk = &a.tk[r];
+      const CUtensorMap* mv = &a.tv[r];
+      tma_prefetch_desc(mq);
+      tma_prefetch_desc(mk);
+      tma_prefetch_desc(mv);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (!active[t]) continue;
+        mbar_arrive_expect_tx(q_full(t), L::kQTile);
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf)
+          tma_load_2d(sQ + t * L::kQTile + hf * (BM * 128), mq, q_full(t), h * D + hf * 64, first_row[t]);
+      }
+      uint32_t it = 0;
+      bool ok = true;
+      for (int jb = jb_lo; jb < jb_hi && ok; ++jb) {
+#pragma unroll
+        for (int kind = 0; kind < 2; ++kind, ++it) {
+          const int s = it % NSTAGE;
+          const uint32_t ph = (it / NSTAGE) & 1u;
+          if (!mbar_wait(kv_empty(s), ph ^ 1u, kErrFwd, 0x100 + s)) { ok = false; break; }
+          mbar_arrive_expect_tx(kv_full(s), L::kKV);
+          const CUtensorMap* m = kind == 0 ? mk : mv;
+#pragma unroll
+          for (int hf = 0; hf < D / 64; ++hf)
+            tma_load_2d(sRing + s * L::kKV + hf * (BN * 128), m, kv_full(s), g * D + hf * 64, jb * BN);
+        }
+      }
+      // Drain: every issued load must land before the CTA can exit.
+      const uint32_t issued = it;
+      for (uint32_t k = issued > NSTAGE ? issued - NSTAGE : 0; k < issued; ++k)
+        mbar_wait(kv_full(k % NSTAGE), (k / NSTAGE) & 1u, kErrFwd, 0x200);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        if (active[t]) mbar_wait(q_full(t), 0, kErrFwd, 0x210 + t);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
+      constexpr uint32_t idO = idesc_bf16_f32(BM, D, 0, 1);
+      bool ok = true;
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        if (active[t] && !mbar_wait(q_full(t), 0, kErrFwd, 0x300 + t)) ok = false;
+      uint32_t it = 0;
+      int cnt[2] = {0, 0};
+      for (int jb = jb_lo; jb < jb_hi && ok; ++jb) {
+        // K block -> S tiles
+        {
+          const int s = it % NSTAGE;
+          const uint32_t ph = (it / NSTAGE) & 1u;
+          ++it;
+          if (!mbar_wait(kv_full(s), ph, kErrFwd, 0x310)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kb = sRing + s * L::kKV;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!active[t] || jb < jb_begin[t] || jb >= jb_end[t]) continue;
+            if (cnt[t] > 0) {
+              if (!mbar_wait(pv_done(t), (cnt[t] - 1) & 1, kErrFwd, 0x320 + t)) { ok = false; break; }
+              tc_fence_after();
+            }
+            const uint32_t qb = sQ + t * L::kQTile;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk / 4) * (BM * 128) + (kk % 4) * 32;
+              const uint64_t ad = smem_desc_sw128(qb + off, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(kb + (kk / 4) * (BN * 128) + (kk % 4) * 32, 16, 1024);
+              mma_ss(tS[t], ad, bd, idS, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(s_full(t));
+          }
+          if (!ok) break;
+          mma_commit(kv_empty(s));
+        }
+        // V block -> O tiles
+        {
+          const int s = it % NSTAGE;
+          const uint32_t ph = (it / NSTAGE) & 1u;
+          ++it;
+          if (!mbar_wait(kv_full(s), ph, kErrFwd, 0x330)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t vb = sRing + s * L::kKV;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!active[t] || jb < jb_begin[t] || jb >= jb_end[t]) continue;
+            if (!mbar_wait(p_full(t), cnt[t] & 1, kErrFwd, 0x340 + t)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk) {
+              const uint64_t bd = smem_desc_sw128(vb + kk * (16 * 128), BN * 128, 1024);
+              mma_ts(tO[t], tS[t] + kk * 8, bd, idO, (cnt[t] > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(pv_done(t));
+            ++cnt[t];
+          }
+          if (!ok) break;
+          mma_commit(kv_empty(s));
+        }
+      }
+      // Drain: wait for every MMA issued above before TMEM can be released.
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, kErrFwd, 0x350);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int t = warp >> 2;
+    const int lrow = 32 * (warp & 3) + lane;        // TMEM lane = row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    if (active[t]) {
+      const int i = first_row[t] + lrow;
+      const bool row_ok = i < N;
+      const int st_i = doc_start_of(a.cu, a.num_seqs, min(i, N - 1));
+      const int max_start = doc_start_of(a.cu, a.num_seqs, last_row[t]);
+      const float sl2 = a.scale_log2;
+      float m_run = -INFINITY, l_run = 0.f;
+      int cnt = 0;
+      bool ok = true;
+      for (int jb = jb_begin[t]; jb < jb_end[t]; ++jb, ++cnt) {
+        if (!mbar_wait(s_full(t), cnt & 1, kErrFwd, 0x400 + t)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t v[BN];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c)
+          tmem_ld32(tS[t] + lane_off + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
+        tmem_wait_ld();
+        const int n0 = jb * BN;
+        const bool need_mask = (n0 + BN - 1 > first_row[t]) || (n0 < max_start);
+        float m_blk = -INFINITY;
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c) {
+            const int key = n0 + c;
+            float x = u2f(v[c]) * sl2;
+            x = (key > i || key < st_i) ? -INFINITY : x;
+            v[c] = __float_as_uint(x);
+            m_blk = fmaxf(m_blk, x);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN; ++c) {
+            const float x = u2f(v[c]) * sl2;
+            v[c] = __float_as_uint(x);
+            m_blk = fmaxf(m_blk, x);
+          }
+        }
+        const float m_new = fmaxf(m_run, m_blk);
+        // Rescale decision (warp-uniform: TMEM loads/stores are warp-collective).
+        bool rescale = false;
+        float alpha = 1.f;
+        if (cnt == 0) {
+          m_run = m_new;
+        } else if (__any_sync(0xffffffffu, m_new > m_run + kRescaleThreshold)) {
+          rescale = true;
+          alpha = (m_new > m_run) ? ex2_approx(m_run - m_new) : 1.f;
+          l_run *= alpha;
+          m_run = m_new;
+        }
+        const float base = (m_run == -INFINITY) ? 0.f : m_run;
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float p0 = ex2_approx(u2f(v[c]) - base);
+          const float p1 = ex2_approx(u2f(v[c + 1]) - base);
+          rs += p0 + p1;
+          v[c / 2] = pack_bf16x2(p0, p1);
+        }
+        l_run += rs;
+        tmem_st32(tS[t] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_st32(tS[t] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        if (rescale) {
+          // O still holds the sum over earlier blocks at the old max: scale it
+          // once the previous P.V has landed, before this block's P.V is issued.
+          if (!mbar_wait(pv_done(t), (cnt - 1) & 1, kErrFwd, 0x410 + t)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t ov[32];
+            tmem_ld32(tO[t] + lane_off + c4 * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(u2f(ov[e]) * alpha);
+            tmem_st32(tO[t] + lane_off + c4 * 32, ov);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full(t));
+      }
+      // epilogue: O / l -> bf16, LSE
+      if (ok && cnt > 0 && mbar_wait(pv_done(t), (cnt - 1) & 1, kErrFwd, 0x420 + t)) {
+        tc_fence_after();
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o.p[r]) + (static_cast<int64_t>(i) * a.Hl + h) * D;
+#pragma unroll 1
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+          uint32_t ov[32];
+          tmem_ld32(tO[t] + lane_off + c4 * 32, ov);
+          tmem_wait_ld();
+          uint4 pk[4];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pw[e] = pack_bf16x2(u2f(ov[2 * e]) * inv, u2f(ov[2 * e + 1]) * inv);
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = pk[e];
+          }
+        }
+        if (row_ok) a.lse.p[r][static_cast<int64_t>(h) * N + i] = (m_run + lg2_approx(l_run)) * kLn2;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D map over a [rows, row_elems] bf16 matrix with 128-byte-swizzled 64 x 128 boxes.
+bool encode_rows(EncodeTiledFn enc, CUtensorMap* m, const void* base, int64_t rows, int64_t row_elems) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_elems), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_elems * 2)};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_d(const FwdArgs& a, int nranks, cudaStream_t stream) {
+  using L = Layout<D>;
+  cudaError_t e =
+      cudaFuncSetAttribute(attn_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.Hl * nranks, a.num_m_blocks);
+  attn_fwd_sm100_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace fwd_sm100
+
+cudaError_t launch_attn_fwd(const AttnShape& s, const void* const* q, const void* const* k, const void* const* v,
+                            void* const* o, float* const* lse, cudaStream_t stream) {
+  using namespace fwd_sm100;
+  EncodeTiledFn enc = get_encode();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  FwdArgs a;   // ~6.5 KB, copied into the launch's parameter space
+  memset(&a, 0, sizeof(a));
+  for (int r = s.rank_lo; r < s.rank_hi; ++r) {
+    if (!encode_rows(enc, &a.tq[r], q[r], s.N, static_cast<int64_t>(s.Hl) * s.d) ||
+        !encode_rows(enc, &a.tk[r], k[r], s.N, static_cast<int64_t>(s.Hkvl) * s.d) ||
+        !encode_rows(enc, &a.tv[r], v[r], s.N, static_cast<int64_t>(s.Hkvl) * s.d))
+      return cudaErrorInvalidValue;
+    a.o.p[r] = o[r];
+    a.lse.p[r] = lse[r];
+  }
+  a.cu = s.cu_seqlens;
+  a.num_seqs = s.num_seqs;
+  a.N = s.N;
+  a.Hl = s.Hl;
+  a.Hkvl = s.Hkvl;
+  a.group = s.Hl / s.Hkvl;
+  a.scale_log2 = s.scale * kLog2e;
+  a.rank_lo = s.rank_lo;
+  a.num_m_blocks = (s.N + 2 * BM - 1) / (2 * BM);
+  const int nranks = s.rank_hi - s.rank_lo;
+  return s.d == 64 ? launch_d<64>(a, nranks, stream) : launch_d<128>(a, nranks, stream);
+}
+
+}  // namespace uly

@@ -2,6 +2,6 @@
 // library's device-side error word and wait cap without relocatable device code.
 #include <string.h>
 #include "permute.cu"
-#include "attn_fwd_mma.cu"
+#include "attn_fwd_sm100.cu"
 #include "attn_bwd_mma.cu"
 #include "api.cu"
