@@ -188,8 +188,13 @@ def main():
     ap.add_argument("--workload", default="varlen64k", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="draw the workload's recipe at a smaller total N (profiling captures)")
     args = ap.parse_args()
     w = workloads.get(args.workload)
+    if args.tokens is not None:
+        import dataclasses
+        w = dataclasses.replace(w, N=args.tokens)
     if args.impl == "reference":
         return run_reference(args, w)
 

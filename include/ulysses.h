@@ -29,9 +29,9 @@
  *     ULY_ERR_UNSUPPORTED nothing is launched and no memory is touched. A
  *     launch failure returns ULY_ERR_CUDA. Nothing aborts or traps.
  *   - Supported shapes: 1 <= P <= ULY_MAX_RANKS; N % P == 0; H % P == 0;
- *     H_kv % P == 0 (the pages' "num_heads >= sp_size", strengthened so that
- *     heads split evenly -- contenidos2-1ml.pages.dev, "¿Qué cambia en la
- *     práctica...?"); H % H_kv == 0; d in {64, 128}; N/P*H*d < 2^31.
+ *     H_kv % P == 0 (the pages require at least as many heads as ranks;
+ *     strengthened here so that heads split evenly -- contenidos2-1ml.pages.dev,
+ *     "¿Qué cambia en la práctica...?"); H % H_kv == 0; d in {64, 128}; N/P*H*d < 2^31.
  *   - cu_seqlens: DEVICE int32 array [num_seqs+1], cu_seqlens[0] = 0,
  *     non-decreasing, cu_seqlens[num_seqs] = N (packed variable-length
  *     documents, block-diagonal causal mask). NULL = one causal sequence.
@@ -65,8 +65,9 @@ typedef enum {
   ULY_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up (see get_device_status) */
 } uly_status;
 
-/* All-to-all #1, sequence sharding -> head sharding (theaicatchup.com, "How Does
- * Ulysses...": "every GPU ends up with all positions, but only a slice of heads").
+/* All-to-all #1, sequence sharding -> head sharding: afterwards each rank holds
+ * the whole sequence for its subset of heads (theaicatchup.com, "How Does
+ * Ulysses Sequence Parallelism Actually Work?").
  *   dst[q][t, j, :] = src[t / (N/P)][t % (N/P), q*Hx/P + j, :]
  * Up to three tensors move in one launch: slot 0 has H heads (Q, or dO in the
  * backward), slots 1 and 2 have H_kv heads (K, V). A NULL slot-1/2 array skips
@@ -82,8 +83,8 @@ ULY_API uly_status ulysses_a2a_seq_to_head(
     int rank_lo, int rank_hi, cudaStream_t stream);
 
 /* All-to-all #2, head sharding -> sequence sharding: the exact inverse of
- * ulysses_a2a_seq_to_head ("Reverse the shuffle", theaicatchup.com, ibid.;
- * "Reconstrução Contextual", radardeia.com).
+ * ulysses_a2a_seq_to_head: after attention the first exchange is undone
+ * (theaicatchup.com, ibid.; radardeia.com, "Arquitetura Técnica").
  *   dst[p][s, q*Hx/P + j, :] = src[q][p*N/P + s, j, :]
  * Slot 0: H heads (O; dQ in the backward); slots 1, 2: H_kv heads (dK, dV).
  * Only SOURCE ranks q in [rank_lo, rank_hi) are read, i.e. only their head
@@ -96,8 +97,8 @@ ULY_API uly_status ulysses_a2a_head_to_seq(
     int rank_lo, int rank_hi, cudaStream_t stream);
 
 /* Causal (optionally packed-varlen) grouped-query flash attention forward on the
- * head shards of ranks [rank_lo, rank_hi) ("Compute attention locally",
- * theaicatchup.com, ibid.; heads are independent, ibid., quoting DeepSpeed-Ulysses):
+ * head shards of ranks [rank_lo, rank_hi): each rank runs attention by itself on
+ * its heads, which do not interact (theaicatchup.com, ibid., citing DeepSpeed-Ulysses):
  *   s_ij = softmax_scale * q_i.k_j  for j <= i in the same document,
  *   o_i = sum_j softmax_j(s_i) v_j  (bf16, round to nearest even),
  *   lse_i = ln sum_j exp(s_ij)      (float32, layout [H/P, N]).
@@ -113,8 +114,10 @@ ULY_API uly_status ulysses_attn_fwd(
     float softmax_scale, int causal,
     int rank_lo, int rank_hi, cudaStream_t stream);
 
-/* Bytes of device workspace ulysses_attn_bwd needs for these sizes (fp32 dQ
- * accumulator and the per-row D_i = dO_i . O_i), for all P ranks. */
+/* Bytes of device workspace ulysses_attn_bwd needs for these sizes: per
+ * (rank, query head, row padded to a multiple of 128) the fp32 values
+ * lse_i*log2(e) and D_i = dO_i . O_i, for all P ranks. Returns 0 for an
+ * invalid shape. */
 ULY_API size_t ulysses_attn_bwd_workspace_size(int64_t N, int P, int H, int H_kv, int d);
 
 /* Attention backward on the head shards of ranks [rank_lo, rank_hi). The pages
@@ -149,8 +152,16 @@ ULY_API const char* ulysses_status_string(uly_status s);
 ULY_API uly_status ulysses_get_device_status(cudaStream_t stream, uint32_t* detail);
 
 /* Test hook: caps every bounded device-side wait at `iters` polls (0 restores
- * the default). Lets a host test make a wait run out without faulting the GPU. */
+ * the default). Waits that drain a CTA before it exits always keep the default
+ * cap. Synchronous; applies to the current device. */
 ULY_API void ulysses_set_wait_limit(uint32_t iters);
+
+/* Test hook: launches one tiny kernel on `stream` that waits, bounded, on an
+ * mbarrier nothing arrives on (the same wait routine the attention kernels use),
+ * so the wait runs out and records kernel id 0x7F, site 0xABC in the device
+ * error word. Nothing faults, traps or hangs; read the result with
+ * ulysses_get_device_status(). Use ulysses_set_wait_limit() first to keep it short. */
+ULY_API uly_status ulysses_selftest_bounded_wait(cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -1,11 +1,10 @@
 """fp64 causal softmax attention, forward and backward (test infrastructure only).
 
-What it computes (per head; the method runs "standard attention" on each head
-independently because "attention heads are independent -- each head can be
-computed separately", theaicatchup.com, quoting the DeepSpeed-Ulysses paper in
-"How Does Ulysses Sequence Parallelism Actually Work?"; Ulysses "no cambia la
-matemática fundamental del attention", contenidos2-1ml.pages.dev,
-"Conclusión rápida"):
+What it computes (per head: the method runs ordinary attention on each head by
+itself, since the heads do not interact -- theaicatchup.com, citing the
+DeepSpeed-Ulysses paper in "How Does Ulysses Sequence Parallelism Actually
+Work?"; the Spanish note stresses that Ulysses leaves the attention arithmetic
+itself unchanged -- contenidos2-1ml.pages.dev, "Conclusión rápida"):
 
   s_ij  = scale * (q_i . k_j)            for allowed j, scale = 1/sqrt(d)
   allowed(i, j)  <=>  j <= i  and  doc(j) == doc(i)

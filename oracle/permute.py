@@ -1,10 +1,10 @@
 """The Ulysses all-to-alls as index arithmetic (test infrastructure only).
 
-Method: before attention, an all-to-all leaves "every GPU with all positions,
-but only a slice of heads"; after attention the shuffle is reversed
+Method: before attention an all-to-all gives each rank the whole sequence for
+a subset of the heads; after attention a second all-to-all undoes it
 (theaicatchup.com, "How Does Ulysses Sequence Parallelism Actually Work?";
-the Spanish note calls them "dos operaciones all-to-all por capa",
-contenidos2-1ml.pages.dev, "¿Qué es Ulysses y por qué importa?").
+two all-to-alls per layer also in contenidos2-1ml.pages.dev, "¿Qué es Ulysses
+y por qué importa?").
 
 Layouts (the pages fix none; plainest reading):
   sequence shard of rank p : [N/P, Hx, d], global token t = p*N/P + s

@@ -95,15 +95,21 @@ def test_softmax_scale_argument():
 
 
 def test_large_logits_stay_finite_and_exact():
-    """Inputs scaled by 4 give scores of magnitude up to ~50: the online softmax
-    must rescale without overflow."""
+    """Inputs scaled by 4 give scores of magnitude up to ~50 and gradients up to
+    ~300: the online softmax must rescale without overflow. At these magnitudes
+    the bf16 rounding of P and dS (relative 2^-9) dominates, so the bar here is
+    relative to each tensor's range: rel RMS <= 1e-2 and max error <= 1% of max|ref|."""
     N, P, H, H_kv, d = 256, 2, 4, 2, 128
     q, k, v, do = _draw(N, H, H_kv, d, seed=11, scale=4.0)
     gpu = run_gpu_layer(q, k, v, do, P, [0, 100, 256])
-    assert np.all(np.isfinite(gpu["o"])) and np.all(np.isfinite(gpu["dq"]))
+    for n in ("o", "dq", "dk", "dv"):
+        assert np.all(np.isfinite(gpu[n])), n
     ref = oracle_layer(q, k, v, do, P, [0, 100, 256])
-    assert_close("O", gpu["o"], ref["o"])
-    assert_close("dV", gpu["dv"], ref["dv"])
+    for r, (a, b) in enumerate(zip(gpu["lse"], ref["lse"])):
+        assert err_stats(a, b)[0] <= LSE_MAX_ABS
+    for n in ("o", "dq", "dk", "dv"):
+        ma, rr = err_stats(gpu[n], ref[n])
+        assert rr <= 1e-2 and ma <= 1e-2 * np.abs(ref[n]).max(), (n, ma, rr)
 
 
 def test_first_token_of_each_document_is_its_value_row():
@@ -120,8 +126,9 @@ def test_first_token_of_each_document_is_its_value_row():
 
 
 def test_result_does_not_depend_on_P():
-    """Heads are independent: P = 1, 2, 4 give bit-identical O, LSE, dK, dV
-    (dQ is summed with atomics in arbitrary order: within tolerance)."""
+    """Heads are independent: P = 1, 2, 4 give bit-identical O, LSE, dQ, dK, dV
+    (the kernels' tiling and summation order do not depend on P, and the
+    backward uses no atomics)."""
     N, H, H_kv, d = 256, 8, 4, 128
     cu = [0, 90, 256]
     q, k, v, do = _draw(N, H, H_kv, d, seed=17)
@@ -131,7 +138,7 @@ def test_result_does_not_depend_on_P():
         assert np.array_equal(g["o"], base["o"])
         assert np.array_equal(np.concatenate(g["lse"], axis=0), base["lse"][0])
         assert np.array_equal(g["dk"], base["dk"]) and np.array_equal(g["dv"], base["dv"])
-        assert_close("dQ", g["dq"], base["dq"], max_abs=1e-2, rel_rms=1e-3)
+        assert np.array_equal(g["dq"], base["dq"])
 
 
 def test_rank_sequential_forward_matches_all_ranks():

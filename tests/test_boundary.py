@@ -63,7 +63,7 @@ def _fwd(L, N=256, P=2, H=8, H_kv=8, d=64, ptr=GOOD, causal=1, lo=0, hi=None, cu
 @pytest.mark.parametrize("kw,code", [
     (dict(P=0), 1), (dict(N=0), 1), (dict(N=255), 1),             # N % P
     (dict(H=8, H_kv=3, P=1), 1),                                   # H % H_kv
-    (dict(P=16, N=256, H=8, H_kv=8), 1),                           # H < P  (num_heads >= sp_size)
+    (dict(P=16, N=256, H=8, H_kv=8), 1),                           # fewer heads than ranks
     (dict(H=8, H_kv=2, P=4), 1),                                   # H_kv % P: kv heads must split too
     (dict(P=17, N=17 * 16, H=17, H_kv=17), 2),                     # more ranks than supported
     (dict(d=96), 2), (dict(d=256), 2),                             # head dims not built
@@ -92,7 +92,7 @@ def test_a2a_validation(L):
 
 def test_bwd_validation_and_workspace_size(L):
     ws = L.ulysses_attn_bwd_workspace_size(8192, 4, 32, 8, 128)
-    assert ws >= 4 * 8192 * 8 * 128 * 4 + 4 * 8192 * 8 * 4
+    assert ws >= 2 * 4 * 8 * 8192 * 4          # lse*log2(e) and D_i per (rank, head, row)
     assert L.ulysses_attn_bwd_workspace_size(8192, 3, 32, 8, 128) == 0     # invalid shape -> 0
     P = 2
     p = _arr([GOOD] * P)

@@ -289,7 +289,7 @@ def test_permute_rank_range_selects_destinations():
 
 
 def test_head_shard_holds_all_positions_for_a_slice_of_heads():
-    """'Every GPU ends up with all positions, but only a slice of heads.'"""
+    """After the first all-to-all a rank holds every token of its own head subset."""
     N, H, d, P = 8, 4, 2, 2
     x = _rand((N, H, d), 46)
     xh = oracle.seq_to_head(workloads.seq_shards(x, P))

@@ -40,6 +40,7 @@ _SIGS = {
     "ulysses_status_string": [_i],
     "ulysses_get_device_status": [_v, ctypes.POINTER(ctypes.c_uint32)],
     "ulysses_set_wait_limit": [ctypes.c_uint32],
+    "ulysses_selftest_bounded_wait": [_v],
 }
 _RES = {"ulysses_attn_bwd_workspace_size": ctypes.c_size_t, "ulysses_status_string": ctypes.c_char_p,
         "ulysses_set_wait_limit": None}

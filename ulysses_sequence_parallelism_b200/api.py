@@ -19,7 +19,8 @@ from ._lib import lib, check, UlyssesError, MAX_RANKS
 
 __all__ = [
     "ulysses_a2a_seq_to_head", "ulysses_a2a_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_bwd",
-    "ulysses_attn_bwd_workspace_size", "ulysses_get_device_status", "ulysses_set_wait_limit", "UlyssesLayer",
+    "ulysses_attn_bwd_workspace_size", "ulysses_get_device_status", "ulysses_set_wait_limit",
+    "ulysses_selftest_bounded_wait", "UlyssesLayer",
 ]
 
 
@@ -109,6 +110,10 @@ def ulysses_get_device_status(stream=None):
 
 def ulysses_set_wait_limit(iters: int):
     lib().ulysses_set_wait_limit(int(iters))
+
+
+def ulysses_selftest_bounded_wait(stream=None):
+    check("ulysses_selftest_bounded_wait", lib().ulysses_selftest_bounded_wait(_stream(stream)))
 
 
 class UlyssesLayer:

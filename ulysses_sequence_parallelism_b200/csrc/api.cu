@@ -7,7 +7,23 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 #include "ulysses.h"
+
+namespace uly {
+// Waits (bounded) on an mbarrier that nothing ever arrives on: exercises the
+// same give-up path as the attention kernels, without touching a real workload.
+__global__ void selftest_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(b, 1);
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) sm100::mbar_wait(b, 0, 0x7Fu, 0xABC);
+}
+}  // namespace uly
 
 namespace {
 
@@ -160,5 +176,10 @@ uly_status ulysses_get_device_status(cudaStream_t stream, uint32_t* detail) {
 }
 
 void ulysses_set_wait_limit(uint32_t iters) { cudaMemcpyToSymbol(uly::g_wait_limit, &iters, sizeof(iters)); }
+
+uly_status ulysses_selftest_bounded_wait(cudaStream_t stream) {
+  uly::selftest_wait_kernel<<<1, 32, 0, stream>>>();
+  return from_cuda(cudaGetLastError());
+}
 
 }  // extern "C"

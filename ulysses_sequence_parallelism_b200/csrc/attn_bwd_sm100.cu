@@ -1,0 +1,725 @@
+// Causal GQA (packed-varlen) flash-attention backward for sm_100a: tcgen05 MMA
+// with TMEM accumulators, TMA-fed shared-memory tiles, warp-specialised.
+//
+// Gradient of the forward (the pages train through the layer but do not write
+// its backward; this is softmax-attention calculus), with scale = softmax scale:
+//   P_ij = exp(s_ij - lse_i),  D_i = dO_i . O_i
+//   dV_j = sum_i P_ij dO_i,    dP_ij = dO_i . v_j,   dS_ij = P_ij (dP_ij - D_i)
+//   dK_j = scale sum_i dS_ij q_i,   dQ_i = scale sum_j dS_ij k_j
+// dK/dV of a key/value head are summed over the H/H_kv query heads reading it.
+//
+// Three launches, deterministic (no atomics anywhere):
+//  1. prep : D_i and lse_i*log2(e) per (rank, head, row) into a workspace
+//            padded to a multiple of 128 rows (padding: lse = +inf, D = 0, so
+//            padded rows contribute exactly zero).
+//  2. dkdv : one CTA per 128-key block of one key/value head. K and V stay in
+//            shared memory; the CTA streams 64-row blocks of Q and dO (every
+//            query head of the group, every row that can see these keys):
+//              S^T = K Q^T, dP^T = V dO^T          (SS MMAs, double-buffered)
+//              P^T, dS^T elementwise (one thread per key row), bf16 into TMEM
+//              dV += P^T dO,  dK += dS^T Q         (TS MMAs into TMEM)
+//  3. dq   : one CTA per 128-row block of one query head. Q and dO stay in
+//            shared memory; the CTA streams 64-key blocks of K and V:
+//              S = Q K^T, dP = dO V^T; dS elementwise (one thread per row);
+//              dQ += dS K (TS MMA into TMEM).
+// S and dP are recomputed in (3): 7 block GEMMs instead of 5, in exchange for
+// no fp32 atomics, no dQ accumulator traffic and a bit-reproducible result.
+// Warp roles in 2 and 3: warps 0-3 / 4-7 elementwise (ping-pong on the two
+// TMEM buffers), warp 8 TMA producer, warp 9 MMA issuer. Every mbarrier wait
+// is bounded and reports into the library error word.
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace uly {
+namespace bwd_sm100 {
+
+using namespace sm100;
+
+constexpr int kThreads = 320;
+constexpr int kTmaWarp = 8, kMmaWarp = 9;
+constexpr int NST = 4;          // ring stages
+constexpr int SB = 64;          // streamed block (rows in dkdv, keys in dq)
+constexpr int TB = 128;         // stationary block (keys in dkdv, rows in dq)
+constexpr float kLog2e = 1.4426950408889634f;
+
+ULY_DEV float u2f(uint32_t x) { return __uint_as_float(x); }
+
+ULY_DEV void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// ====================================================================== prep
+struct PrepArgs {
+  RankPtrs o, dO;
+  RankPtrsFC lse;
+  float* lse2;    // [P][Hl][Npad]
+  float* Dv;      // [P][Hl][Npad]
+  int N, Npad, Hl, rank_lo, nranks;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ PrepArgs a) {
+  constexpr int CH = D / 8;            // 16-byte chunks per head row
+  constexpr int RPB = 256 / CH;
+  const int64_t rows_per_rank = static_cast<int64_t>(a.Npad) * a.Hl;
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * RPB + threadIdx.x / CH;
+  const int c = threadIdx.x % CH;
+  const bool ok = e < rows_per_rank * a.nranks;
+  int r = 0, i = 0, h = 0;
+  float sum = 0.f;
+  if (ok) {
+    const int rr = static_cast<int>(e / rows_per_rank);
+    const int64_t rem = e - rr * rows_per_rank;
+    i = static_cast<int>(rem / a.Hl);
+    h = static_cast<int>(rem - static_cast<int64_t>(i) * a.Hl);
+    r = a.rank_lo + rr;
+    if (i < a.N) {
+      const int64_t off = (static_cast<int64_t>(i) * a.Hl + h) * D + c * 8;
+      const uint4 ov = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o.p[r]) + off);
+      const uint4 dv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dO.p[r]) + off);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+      const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 of = __bfloat1622float2(o2[k]);
+        const float2 df = __bfloat1622float2(d2[k]);
+        sum = fmaf(of.x, df.x, sum);
+        sum = fmaf(of.y, df.y, sum);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = CH / 2; m >= 1; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
+  if (ok && c == 0) {
+    const int64_t idx = (static_cast<int64_t>(r) * a.Hl + h) * a.Npad + i;
+    if (i < a.N) {
+      a.Dv[idx] = sum;
+      a.lse2[idx] = a.lse.p[r][static_cast<int64_t>(h) * a.N + i] * kLog2e;
+    } else {
+      a.Dv[idx] = 0.f;
+      a.lse2[idx] = INFINITY;
+    }
+  }
+}
+
+// ====================================================================== dK, dV
+struct DkdvArgs {
+  CUtensorMap tq[kMaxRanks];    // box 64 cols x SB rows
+  CUtensorMap tdo[kMaxRanks];   // box 64 cols x SB rows
+  CUtensorMap tk[kMaxRanks];    // box 64 cols x TB rows
+  CUtensorMap tv[kMaxRanks];    // box 64 cols x TB rows
+  RankPtrsMut dk, dv;
+  const float* lse2;
+  const float* Dv;
+  const int32_t* cu;
+  int num_seqs;
+  int N, Npad, Hl, Hkvl, group;
+  float scale, scale_log2;
+  int rank_lo;
+};
+
+template <int D>
+struct DkdvLayout {
+  static constexpr uint32_t kKV = TB * D * 2;         // one stationary K or V tile
+  static constexpr uint32_t kBlk = SB * D * 2;        // one streamed Q or dO block
+  static constexpr uint32_t kK = 0, kV = kKV;
+  static constexpr uint32_t kRing = 2 * kKV;          // stage s: Q at +0, dO at +kBlk
+  static constexpr uint32_t kVec = kRing + NST * 2 * kBlk;   // stage s: lse2 at +0, D at +256
+  static constexpr uint32_t kBars = kVec + NST * 512;
+  // kv_full, st_full[NST], st_empty[NST], s_full[2], dp_full[2], p_full[2], ds_full[2], buf_free[2], acc_done
+  static constexpr int kNumBars = 1 + 2 * NST + 10 + 1;
+  static constexpr uint32_t kSlot = kBars + kNumBars * 8;
+  static constexpr uint32_t kAlloc = kSlot + 16 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid_constant__ DkdvArgs a) {
+  using L = DkdvLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  const uint32_t bars = sbase + L::kBars;
+  const uint32_t kv_full = bars;
+  auto st_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto st_empty = [&](int s) { return bars + 8u * (1 + NST + s); };
+  auto s_full = [&](int b) { return bars + 8u * (1 + 2 * NST + b); };
+  auto dp_full = [&](int b) { return bars + 8u * (3 + 2 * NST + b); };
+  auto p_full = [&](int b) { return bars + 8u * (5 + 2 * NST + b); };
+  auto ds_full = [&](int b) { return bars + 8u * (7 + 2 * NST + b); };
+  auto buf_free = [&](int b) { return bars + 8u * (9 + 2 * NST + b); };
+  const uint32_t acc_done = bars + 8u * (11 + 2 * NST);
+  volatile uint32_t* slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kSlot);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.x % a.Hkvl;
+  const int r = a.rank_lo + blockIdx.x / a.Hkvl;
+  const int N = a.N;
+  const int n0 = blockIdx.y * TB;                      // key blocks near the start carry the most rows
+  const int n_last = min(n0 + TB, N) - 1;
+  const int doc_end_first = doc_end_of(a.cu, a.num_seqs, n0, N);
+  const int m_end = doc_end_of(a.cu, a.num_seqs, n_last, N);
+  const int rb_lo = n0 / SB;
+  const int nrb = (m_end + SB - 1) / SB - rb_lo;
+  const int T = a.group * nrb;                          // streamed iterations
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::kNumBars; ++i) mbar_init(bars + 8u * i, 1);
+    mbar_init(p_full(0), 128);
+    mbar_init(p_full(1), 128);
+    mbar_init(ds_full(0), 128);
+    mbar_init(ds_full(1), 128);
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(sbase + L::kSlot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  const uint32_t tDV = tmem, tDK = tmem + D;
+  auto tS = [&](int b) { return tmem + 256u + 128u * b; };
+  auto tDP = [&](int b) { return tmem + 256u + 128u * b + 64u; };
+
+  if (warp == kTmaWarp) {
+    if (lane == 0) {
+      const CUtensorMap *mq = &a.tq[r], *mdo = &a.tdo[r], *mk = &a.tk[r], *mv = &a.tv[r];
+      tma_prefetch_desc(mq);
+      tma_prefetch_desc(mdo);
+      mbar_arrive_expect_tx(kv_full, 2 * L::kKV);
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf) {
+        tma_load_2d(sbase + L::kK + hf * (TB * 128), mk, kv_full, g * D + hf * 64, n0);
+        tma_load_2d(sbase + L::kV + hf * (TB * 128), mv, kv_full, g * D + hf * 64, n0);
+      }
+      int it = 0;
+      for (; it < T; ++it) {
+        const int s = it % NST;
+        if (!mbar_wait(st_empty(s), ((it / NST) & 1) ^ 1, kErrBwd, 0x100 + s)) break;
+        const int h = g * a.group + it / nrb;
+        const int m0 = (rb_lo + it % nrb) * SB;
+        const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
+        mbar_arrive_expect_tx(st_full(s), 2 * L::kBlk + 512);
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf) {
+          tma_load_2d(stg + hf * (SB * 128), mq, st_full(s), h * D + hf * 64, m0);
+          tma_load_2d(stg + L::kBlk + hf * (SB * 128), mdo, st_full(s), h * D + hf * 64, m0);
+        }
+        const int64_t vo = (static_cast<int64_t>(r) * a.Hl + h) * a.Npad + m0;
+        bulk_load(sbase + L::kVec + s * 512, a.lse2 + vo, SB * 4, st_full(s));
+        bulk_load(sbase + L::kVec + s * 512 + 256, a.Dv + vo, SB * 4, st_full(s));
+      }
+      for (int k = it > NST ? it - NST : 0; k < it; ++k)
+        mbar_wait_drain(st_full(k % NST), (k / NST) & 1, kErrBwd, 0x1f0);
+      mbar_wait_drain(kv_full, 0, kErrBwd, 0x1f1);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(TB, SB, 0, 0);
+      constexpr uint32_t idA = idesc_bf16_f32(TB, D, 0, 1);
+      bool ok = mbar_wait(kv_full, 0, kErrBwd, 0x200);
+      tc_fence_after();
+      auto issue_sdp = [&](int it) -> bool {
+        const int b = it & 1, s = it % NST;
+        if (!mbar_wait(st_full(s), (it / NST) & 1, kErrBwd, 0x210)) return false;
+        if (it >= 2 && !mbar_wait(buf_free(b), ((it - 2) >> 1) & 1, kErrBwd, 0x220)) return false;
+        tc_fence_after();
+        const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk / 4) * (TB * 128) + (kk % 4) * 32;
+          const uint32_t qo = (kk / 4) * (SB * 128) + (kk % 4) * 32;
+          mma_ss(tS(b), smem_desc_sw128(sbase + L::kK + ko, 16, 1024), smem_desc_sw128(stg + qo, 16, 1024), idS,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full(b));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk / 4) * (TB * 128) + (kk % 4) * 32;
+          const uint32_t qo = (kk / 4) * (SB * 128) + (kk % 4) * 32;
+          mma_ss(tDP(b), smem_desc_sw128(sbase + L::kV + ko, 16, 1024),
+                 smem_desc_sw128(stg + L::kBlk + qo, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(dp_full(b));
+        return true;
+      };
+      auto issue_acc = [&](int it) -> bool {
+        const int b = it & 1, s = it % NST;
+        const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
+        if (!mbar_wait(p_full(b), (it >> 1) & 1, kErrBwd, 0x230)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < SB / 16; ++kk)
+          mma_ts(tDV, tS(b) + kk * 8, smem_desc_sw128(stg + L::kBlk + kk * 2048, SB * 128, 1024), idA,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        if (!mbar_wait(ds_full(b), (it >> 1) & 1, kErrBwd, 0x240)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < SB / 16; ++kk)
+          mma_ts(tDK, tDP(b) + kk * 8, smem_desc_sw128(stg + kk * 2048, SB * 128, 1024), idA,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(st_empty(s));
+        mma_commit(buf_free(b));
+        return true;
+      };
+      if (ok && T > 0) ok = issue_sdp(0);
+      for (int it = 0; it < T && ok; ++it) {
+        if (it + 1 < T && !issue_sdp(it + 1)) { ok = false; break; }
+        ok = issue_acc(it);
+      }
+      mma_commit(acc_done);
+      mbar_wait_drain(acc_done, 0, kErrBwd, 0x250);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ elementwise
+    const int b = warp >> 2;                            // this warpgroup's TMEM buffer
+    const int lrow = 32 * (warp & 3) + lane;            // TMEM lane = key row
+    const uint32_t loff = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const int key = n0 + lrow;
+    const int kde = doc_end_of(a.cu, a.num_seqs, min(key, N - 1), N);   // rows allowed: key <= row < kde
+    const float sl2 = a.scale_log2;
+    bool ok = true;
+    for (int it = b; it < T; it += 2) {
+      const int s = it % NST;
+      const int m0 = (rb_lo + it % nrb) * SB;
+      const float* vl = reinterpret_cast<const float*>(sgen + L::kVec + s * 512);
+      const float* vd = vl + 64;
+      if (!mbar_wait_warp(st_full(s), (it / NST) & 1, kErrBwd, 0x300)) { ok = false; break; }
+      if (!mbar_wait_warp(s_full(b), (it >> 1) & 1, kErrBwd, 0x310)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t pv[SB];
+      tmem_ld32(tS(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
+      tmem_ld32(tS(b) + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
+      tmem_wait_ld();
+      const bool need_mask = (m0 < n0 + TB - 1) || (m0 + SB > doc_end_first);
+      uint32_t pk[SB / 2];
+#pragma unroll
+      for (int c = 0; c < SB; ++c) {
+        const int row = m0 + c;
+        float p = ex2_approx(u2f(pv[c]) * sl2 - vl[c]);
+        if (need_mask && (row < key || row >= kde)) p = 0.f;
+        pv[c] = __float_as_uint(p);
+      }
+#pragma unroll
+      for (int c = 0; c < SB / 2; ++c) pk[c] = pack_bf16x2(u2f(pv[2 * c]), u2f(pv[2 * c + 1]));
+      tmem_st32(tS(b) + loff, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full(b));
+      if (!mbar_wait_warp(dp_full(b), (it >> 1) & 1, kErrBwd, 0x320)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t dp[32];
+        tmem_ld32(tDP(b) + loff + half * 32, dp);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int c0 = half * 32 + 2 * c;
+          const float d0 = u2f(pv[c0]) * (u2f(dp[2 * c]) - vd[c0]);
+          const float d1 = u2f(pv[c0 + 1]) * (u2f(dp[2 * c + 1]) - vd[c0 + 1]);
+          pk[half * 16 + c] = pack_bf16x2(d0, d1);
+        }
+      }
+      tmem_st32(tDP(b) + loff, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(ds_full(b));
+    }
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes scale * dK
+    if (ok && mbar_wait_warp(acc_done, 0, kErrBwd, 0x330)) {
+      tc_fence_after();
+      const uint32_t src = (b == 0 ? tDV : tDK) + loff;
+      const float mul = b == 0 ? 1.f : a.scale;
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(b == 0 ? a.dv.p[r] : a.dk.p[r]) +
+                           (static_cast<int64_t>(key) * a.Hkvl + g) * D;
+#pragma unroll 1
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t v[32];
+        tmem_ld32(src + c4 * 32, v);
+        tmem_wait_ld();
+        uint4 o4[4];
+        uint32_t* ow = reinterpret_cast<uint32_t*>(o4);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) ow[e] = pack_bf16x2(u2f(v[2 * e]) * mul, u2f(v[2 * e + 1]) * mul);
+        if (key < N) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c4 * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d4[e] = o4[e];
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ====================================================================== dQ
+struct DqArgs {
+  CUtensorMap tq[kMaxRanks];    // box 64 cols x TB rows
+  CUtensorMap tdo[kMaxRanks];   // box 64 cols x TB rows
+  CUtensorMap tk[kMaxRanks];    // box 64 cols x SB rows
+  CUtensorMap tv[kMaxRanks];    // box 64 cols x SB rows
+  RankPtrsMut dq;
+  const float* lse2;
+  const float* Dv;
+  const int32_t* cu;
+  int num_seqs;
+  int N, Npad, Hl, Hkvl, group;
+  float scale, scale_log2;
+  int rank_lo;
+  int num_m_tiles;
+};
+
+template <int D>
+struct DqLayout {
+  static constexpr uint32_t kTile = TB * D * 2;
+  static constexpr uint32_t kBlk = SB * D * 2;
+  static constexpr uint32_t kQ = 0, kDO = kTile;
+  static constexpr uint32_t kRing = 2 * kTile;        // stage s: K at +0, V at +kBlk
+  static constexpr uint32_t kBars = kRing + NST * 2 * kBlk;
+  // q_full, st_full[NST], st_empty[NST], s_full[2], dp_full[2], ds_full[2], buf_free[2], acc_done
+  static constexpr int kNumBars = 1 + 2 * NST + 8 + 1;
+  static constexpr uint32_t kSlot = kBars + kNumBars * 8;
+  static constexpr uint32_t kAlloc = kSlot + 16 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_constant__ DqArgs a) {
+  using L = DqLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  const uint32_t bars = sbase + L::kBars;
+  const uint32_t q_full = bars;
+  auto st_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto st_empty = [&](int s) { return bars + 8u * (1 + NST + s); };
+  auto s_full = [&](int b) { return bars + 8u * (1 + 2 * NST + b); };
+  auto dp_full = [&](int b) { return bars + 8u * (3 + 2 * NST + b); };
+  auto ds_full = [&](int b) { return bars + 8u * (5 + 2 * NST + b); };
+  auto buf_free = [&](int b) { return bars + 8u * (7 + 2 * NST + b); };
+  const uint32_t acc_done = bars + 8u * (9 + 2 * NST);
+  volatile uint32_t* slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kSlot);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x % a.Hl;
+  const int r = a.rank_lo + blockIdx.x / a.Hl;
+  const int g = h / a.group;
+  const int N = a.N;
+  const int m0 = (a.num_m_tiles - 1 - static_cast<int>(blockIdx.y)) * TB;   // longest first
+  const int m_last = min(m0 + TB, N) - 1;
+  const int kb_lo = doc_start_of(a.cu, a.num_seqs, m0) / SB;
+  const int T = m_last / SB + 1 - kb_lo;
+  const int max_start = doc_start_of(a.cu, a.num_seqs, m_last);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::kNumBars; ++i) mbar_init(bars + 8u * i, 1);
+    mbar_init(ds_full(0), 128);
+    mbar_init(ds_full(1), 128);
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(sbase + L::kSlot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  const uint32_t tDQ = tmem;
+  auto tS = [&](int b) { return tmem + 128u + 128u * b; };
+  auto tDP = [&](int b) { return tmem + 128u + 128u * b + 64u; };
+
+  if (warp == kTmaWarp) {
+    if (lane == 0) {
+      const CUtensorMap *mq = &a.tq[r], *mdo = &a.tdo[r], *mk = &a.tk[r], *mv = &a.tv[r];
+      tma_prefetch_desc(mk);
+      tma_prefetch_desc(mv);
+      mbar_arrive_expect_tx(q_full, 2 * L::kTile);
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf) {
+        tma_load_2d(sbase + L::kQ + hf * (TB * 128), mq, q_full, h * D + hf * 64, m0);
+        tma_load_2d(sbase + L::kDO + hf * (TB * 128), mdo, q_full, h * D + hf * 64, m0);
+      }
+      int it = 0;
+      for (; it < T; ++it) {
+        const int s = it % NST;
+        if (!mbar_wait(st_empty(s), ((it / NST) & 1) ^ 1, kErrBwd, 0x500 + s)) break;
+        const int k0 = (kb_lo + it) * SB;
+        const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
+        mbar_arrive_expect_tx(st_full(s), 2 * L::kBlk);
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf) {
+          tma_load_2d(stg + hf * (SB * 128), mk, st_full(s), g * D + hf * 64, k0);
+          tma_load_2d(stg + L::kBlk + hf * (SB * 128), mv, st_full(s), g * D + hf * 64, k0);
+        }
+      }
+      for (int k = it > NST ? it - NST : 0; k < it; ++k)
+        mbar_wait_drain(st_full(k % NST), (k / NST) & 1, kErrBwd, 0x5f0);
+      mbar_wait_drain(q_full, 0, kErrBwd, 0x5f1);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(TB, SB, 0, 0);
+      constexpr uint32_t idA = idesc_bf16_f32(TB, D, 0, 1);
+      bool ok = mbar_wait(q_full, 0, kErrBwd, 0x600);
+      tc_fence_after();
+      auto issue_sdp = [&](int it) -> bool {
+        const int b = it & 1, s = it % NST;
+        if (!mbar_wait(st_full(s), (it / NST) & 1, kErrBwd, 0x610)) return false;
+        if (it >= 2 && !mbar_wait(buf_free(b), ((it - 2) >> 1) & 1, kErrBwd, 0x620)) return false;
+        tc_fence_after();
+        const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qo = (kk / 4) * (TB * 128) + (kk % 4) * 32;
+          const uint32_t ko = (kk / 4) * (SB * 128) + (kk % 4) * 32;
+          mma_ss(tS(b), smem_desc_sw128(sbase + L::kQ + qo, 16, 1024), smem_desc_sw128(stg + ko, 16, 1024), idS,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full(b));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qo = (kk / 4) * (TB * 128) + (kk % 4) * 32;
+          const uint32_t ko = (kk / 4) * (SB * 128) + (kk % 4) * 32;
+          mma_ss(tDP(b), smem_desc_sw128(sbase + L::kDO + qo, 16, 1024),
+                 smem_desc_sw128(stg + L::kBlk + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(dp_full(b));
+        return true;
+      };
+      auto issue_acc = [&](int it) -> bool {
+        const int b = it & 1, s = it % NST;
+        const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
+        if (!mbar_wait(ds_full(b), (it >> 1) & 1, kErrBwd, 0x630)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < SB / 16; ++kk)
+          mma_ts(tDQ, tS(b) + kk * 8, smem_desc_sw128(stg + kk * 2048, SB * 128, 1024), idA,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(st_empty(s));
+        mma_commit(buf_free(b));
+        return true;
+      };
+      if (ok && T > 0) ok = issue_sdp(0);
+      for (int it = 0; it < T && ok; ++it) {
+        if (it + 1 < T && !issue_sdp(it + 1)) { ok = false; break; }
+        ok = issue_acc(it);
+      }
+      mma_commit(acc_done);
+      mbar_wait_drain(acc_done, 0, kErrBwd, 0x640);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ elementwise
+    const int b = warp >> 2;
+    const int lrow = 32 * (warp & 3) + lane;            // TMEM lane = query row
+    const uint32_t loff = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const int i = m0 + lrow;
+    const int ic = min(i, N - 1);
+    const int st_i = doc_start_of(a.cu, a.num_seqs, ic);
+    const int64_t vo = (static_cast<int64_t>(r) * a.Hl + h) * a.Npad + i;   // padded: always in bounds
+    const float lse2_i = a.lse2[vo];
+    const float D_i = a.Dv[vo];
+    const float sl2 = a.scale_log2;
+    bool ok = true;
+    for (int it = b; it < T; it += 2) {
+      const int k0 = (kb_lo + it) * SB;
+      if (!mbar_wait_warp(s_full(b), (it >> 1) & 1, kErrBwd, 0x700)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t pv[SB];
+      tmem_ld32(tS(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
+      tmem_ld32(tS(b) + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
+      tmem_wait_ld();
+      const bool need_mask = (k0 + SB - 1 > m0) || (k0 < max_start);
+#pragma unroll
+      for (int c = 0; c < SB; ++c) {
+        const int key = k0 + c;
+        float p = ex2_approx(u2f(pv[c]) * sl2 - lse2_i);
+        if (need_mask && (key > i || key < st_i)) p = 0.f;
+        pv[c] = __float_as_uint(p);
+      }
+      if (!mbar_wait_warp(dp_full(b), (it >> 1) & 1, kErrBwd, 0x710)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t pk[SB / 2];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t dp[32];
+        tmem_ld32(tDP(b) + loff + half * 32, dp);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int c0 = half * 32 + 2 * c;
+          pk[half * 16 + c] = pack_bf16x2(u2f(pv[c0]) * (u2f(dp[2 * c]) - D_i),
+                                          u2f(pv[c0 + 1]) * (u2f(dp[2 * c + 1]) - D_i));
+        }
+      }
+      tmem_st32(tS(b) + loff, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(ds_full(b));
+    }
+    // epilogue: each warpgroup writes half of the dQ row (columns b*D/2 ...)
+    if (ok && mbar_wait_warp(acc_done, 0, kErrBwd, 0x720)) {
+      tc_fence_after();
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dq.p[r]) + (static_cast<int64_t>(i) * a.Hl + h) * D;
+#pragma unroll 1
+      for (int c4 = b * (D / 64); c4 < (b + 1) * (D / 64); ++c4) {
+        uint32_t v[32];
+        tmem_ld32(tDQ + loff + c4 * 32, v);
+        tmem_wait_ld();
+        uint4 o4[4];
+        uint32_t* ow = reinterpret_cast<uint32_t*>(o4);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) ow[e] = pack_bf16x2(u2f(v[2 * e]) * a.scale, u2f(v[2 * e + 1]) * a.scale);
+        if (i < N) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c4 * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d4[e] = o4[e];
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ====================================================================== host
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool encode(EncodeTiledFn enc, CUtensorMap* m, const void* base, int64_t rows, int64_t row_elems, int box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_elems), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_elems * 2)};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline int padded_rows(int N) { return (N + TB - 1) / TB * TB; }
+
+template <int D>
+cudaError_t launch_all(const AttnShape& s, const PrepArgs& pa, const DkdvArgs& ka, const DqArgs& qa,
+                       cudaStream_t stream) {
+  const int nranks = s.rank_hi - s.rank_lo;
+  {
+    constexpr int RPB = 256 / (D / 8);
+    const int64_t rows = static_cast<int64_t>(pa.Npad) * s.Hl * nranks;
+    bwd_prep_kernel<D><<<static_cast<unsigned>((rows + RPB - 1) / RPB), 256, 0, stream>>>(pa);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  {
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         DkdvLayout<D>::kAlloc);
+    if (e != cudaSuccess) return e;
+    dim3 grid(s.Hkvl * nranks, (s.N + TB - 1) / TB);
+    attn_bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kAlloc, stream>>>(ka);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  {
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         DqLayout<D>::kAlloc);
+    if (e != cudaSuccess) return e;
+    dim3 grid(s.Hl * nranks, qa.num_m_tiles);
+    attn_bwd_dq_kernel<D><<<grid, kThreads, DqLayout<D>::kAlloc, stream>>>(qa);
+    return cudaGetLastError();
+  }
+}
+
+}  // namespace bwd_sm100
+
+size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d) {
+  (void)d;
+  const int64_t npad = (N + bwd_sm100::TB - 1) / bwd_sm100::TB * bwd_sm100::TB;
+  return 2 * static_cast<size_t>(P) * Hl * npad * sizeof(float);
+}
+
+cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void* const* k, const void* const* v,
+                            const void* const* o, const float* const* lse, const void* const* dO, void* const* dq,
+                            void* const* dk, void* const* dv, void* workspace, cudaStream_t stream) {
+  using namespace bwd_sm100;
+  EncodeTiledFn enc = get_encode();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  const int Npad = padded_rows(s.N);
+  float* lse2 = static_cast<float*>(workspace);
+  float* Dv = lse2 + static_cast<size_t>(s.P) * s.Hl * Npad;
+
+  PrepArgs pa;
+  memset(&pa, 0, sizeof(pa));
+  DkdvArgs ka;
+  memset(&ka, 0, sizeof(ka));
+  DqArgs qa;
+  memset(&qa, 0, sizeof(qa));
+  const int64_t qe = static_cast<int64_t>(s.Hl) * s.d, ke = static_cast<int64_t>(s.Hkvl) * s.d;
+  for (int r = s.rank_lo; r < s.rank_hi; ++r) {
+    pa.o.p[r] = o[r];
+    pa.dO.p[r] = dO[r];
+    pa.lse.p[r] = lse[r];
+    if (!encode(enc, &ka.tq[r], q[r], s.N, qe, SB) || !encode(enc, &ka.tdo[r], dO[r], s.N, qe, SB) ||
+        !encode(enc, &ka.tk[r], k[r], s.N, ke, TB) || !encode(enc, &ka.tv[r], v[r], s.N, ke, TB) ||
+        !encode(enc, &qa.tq[r], q[r], s.N, qe, TB) || !encode(enc, &qa.tdo[r], dO[r], s.N, qe, TB) ||
+        !encode(enc, &qa.tk[r], k[r], s.N, ke, SB) || !encode(enc, &qa.tv[r], v[r], s.N, ke, SB))
+      return cudaErrorInvalidValue;
+    ka.dk.p[r] = dk[r];
+    ka.dv.p[r] = dv[r];
+    qa.dq.p[r] = dq[r];
+  }
+  pa.lse2 = lse2;
+  pa.Dv = Dv;
+  pa.N = s.N;
+  pa.Npad = Npad;
+  pa.Hl = s.Hl;
+  pa.rank_lo = s.rank_lo;
+  pa.nranks = s.rank_hi - s.rank_lo;
+
+  ka.lse2 = qa.lse2 = lse2;
+  ka.Dv = qa.Dv = Dv;
+  ka.cu = qa.cu = s.cu_seqlens;
+  ka.num_seqs = qa.num_seqs = s.num_seqs;
+  ka.N = qa.N = s.N;
+  ka.Npad = qa.Npad = Npad;
+  ka.Hl = qa.Hl = s.Hl;
+  ka.Hkvl = qa.Hkvl = s.Hkvl;
+  ka.group = qa.group = s.Hl / s.Hkvl;
+  ka.scale = qa.scale = s.scale;
+  ka.scale_log2 = qa.scale_log2 = s.scale * kLog2e;
+  ka.rank_lo = qa.rank_lo = s.rank_lo;
+  qa.num_m_tiles = (s.N + TB - 1) / TB;
+  return s.d == 64 ? launch_all<64>(s, pa, ka, qa, stream) : launch_all<128>(s, pa, ka, qa, stream);
+}
+
+}  // namespace uly

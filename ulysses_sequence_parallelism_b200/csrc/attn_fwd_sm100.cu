@@ -4,9 +4,9 @@
 // Computes, per rank in range, per local query head h, per row i:
 //   s_ij = scale * q_i.k_j  (j <= i, same document),  o_i = softmax_j(s_i) V,
 //   lse_i = ln sum_j exp(s_ij)
-// ("Compute attention locally" on every rank's head slice over all positions,
-// heads being independent -- theaicatchup.com, "How Does Ulysses Sequence
-// Parallelism Actually Work?").
+// (each rank runs attention by itself on its own heads over the whole
+// sequence, the heads not interacting -- theaicatchup.com, "How Does Ulysses
+// Sequence Parallelism Actually Work?").
 //
 // One CTA owns two 128-row query tiles of one head (256 rows) and streams the
 // 128-key K/V blocks they need through a 4-stage shared-memory ring:
@@ -168,10 +168,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
       // Drain: every issued load must land before the CTA can exit.
       const uint32_t issued = it;
       for (uint32_t k = issued > NSTAGE ? issued - NSTAGE : 0; k < issued; ++k)
-        mbar_wait(kv_full(k % NSTAGE), (k / NSTAGE) & 1u, kErrFwd, 0x200);
+        mbar_wait_drain(kv_full(k % NSTAGE), (k / NSTAGE) & 1u, kErrFwd, 0x200);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-        if (active[t]) mbar_wait(q_full(t), 0, kErrFwd, 0x210 + t);
+        if (active[t]) mbar_wait_drain(q_full(t), 0, kErrFwd, 0x210 + t);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
       }
       // Drain: wait for every MMA issued above before TMEM can be released.
       mma_commit(mma_done);
-      mbar_wait(mma_done, 0, kErrFwd, 0x350);
+      mbar_wait_drain(mma_done, 0, kErrFwd, 0x350);
     }
     __syncwarp();
   } else {
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
       int cnt = 0;
       bool ok = true;
       for (int jb = jb_begin[t]; jb < jb_end[t]; ++jb, ++cnt) {
-        if (!mbar_wait(s_full(t), cnt & 1, kErrFwd, 0x400 + t)) { ok = false; break; }
+        if (!mbar_wait_warp(s_full(t), cnt & 1, kErrFwd, 0x400 + t)) { ok = false; break; }
         tc_fence_after();
         uint32_t v[BN];
 #pragma unroll
@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
         if (rescale) {
           // O still holds the sum over earlier blocks at the old max: scale it
           // once the previous P.V has landed, before this block's P.V is issued.
-          if (!mbar_wait(pv_done(t), (cnt - 1) & 1, kErrFwd, 0x410 + t)) { ok = false; break; }
+          if (!mbar_wait_warp(pv_done(t), (cnt - 1) & 1, kErrFwd, 0x410 + t)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int c4 = 0; c4 < D / 32; ++c4) {
@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
         mbar_arrive(p_full(t));
       }
       // epilogue: O / l -> bf16, LSE
-      if (ok && cnt > 0 && mbar_wait(pv_done(t), (cnt - 1) & 1, kErrFwd, 0x420 + t)) {
+      if (ok && cnt > 0 && mbar_wait_warp(pv_done(t), (cnt - 1) & 1, kErrFwd, 0x420 + t)) {
         tc_fence_after();
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o.p[r]) + (static_cast<int64_t>(i) * a.Hl + h) * D;

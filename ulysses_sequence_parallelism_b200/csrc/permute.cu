@@ -1,9 +1,9 @@
 // Ulysses all-to-all emulation on one GPU: sequence <-> head sharding permutes.
 //
 // The method's two all-to-alls per layer (theaicatchup.com, "How Does Ulysses
-// Sequence Parallelism Actually Work?": shuffle so "every GPU ends up with all
-// positions, but only a slice of heads", then "Reverse the shuffle") become,
-// with the P ranks as P buffers of one GPU, pure index maps:
+// Sequence Parallelism Actually Work?": the first gives each rank the whole
+// sequence for its subset of heads, the second undoes it after attention)
+// become, with the P ranks as P buffers of one GPU, pure index maps:
 //   seq -> head : head[q][t, j, :] = seq[t / n][t % n, q*Hl + j, :]   (n = N/P, Hl = Hx/P)
 //   head -> seq : the inverse.
 // HBM-bound: every byte is read once and written once. The kernel walks the
@@ -22,7 +22,8 @@ namespace permute_impl {
 
 constexpr int kThreads = 512;
 constexpr int kMaxVecPerThread = 8;     // supports Hx*d/8 <= 4096 vectors per row
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 8;
+constexpr int kTargetBlocks = 148 * 8;  // ~2 waves of 4 resident 512-thread blocks per SM
 
 struct SlotArgs {
   RankPtrs src;
@@ -33,6 +34,7 @@ struct SlotArgs {
 
 struct PermuteArgs {
   SlotArgs slot[3];
+  int slot_of[3];  // blockIdx.y / P -> slot (active slots only)
   int n;           // tokens per rank (N/P)
   int P;
   int dvec;        // d / 8 : 16-byte vectors per head row
@@ -53,10 +55,9 @@ ULY_DEV void st_vec(uint4* p, const uint4& v) {
 
 template <bool kSeqToHead>
 __global__ void __launch_bounds__(kThreads) permute_kernel(const __grid_constant__ PermuteArgs a) {
-  const int slot_id = blockIdx.y / a.P;
-  const int p = blockIdx.y - slot_id * a.P;          // sequence-side rank
-  const SlotArgs& sl = a.slot[slot_id];
-  if (!sl.active) return;
+  const int yi = blockIdx.y / a.P;
+  const int p = blockIdx.y - yi * a.P;               // sequence-side rank
+  const SlotArgs& sl = a.slot[a.slot_of[yi]];
   const int Hl = sl.hx / a.P;
   const int row_vecs = sl.hx * a.dvec;                // vectors per sequence-side row
   const int head_row_vecs = Hl * a.dvec;              // vectors per head-side token row
@@ -156,12 +157,12 @@ cudaError_t launch_permute(bool seq_to_head, const void* const* src[3], void* co
   a.rank_lo = rank_lo;
   a.rank_hi = rank_hi;
   int max_rows_per_pass = 1;
-  int any = 0;
+  int n_active = 0;
   for (int s = 0; s < 3; ++s) {
     a.slot[s].active = (src[s] != nullptr && dst[s] != nullptr) ? 1 : 0;
     a.slot[s].hx = hx[s];
     if (!a.slot[s].active) continue;
-    any = 1;
+    a.slot_of[n_active++] = s;
     const bool sr = seq_to_head;
     for (int r = 0; r < P; ++r) {
       // sequence-side buffers: every rank; head-side buffers: ranks in range only.
@@ -174,13 +175,14 @@ cudaError_t launch_permute(bool seq_to_head, const void* const* src[3], void* co
     int rpp = rv <= kThreads ? kThreads / rv : 1;
     if (rpp > max_rows_per_pass) max_rows_per_pass = rpp;
   }
-  if (!any || a.n == 0) return cudaSuccess;
-  // Rows per block: a multiple of every slot's rows-per-pass (all powers of two or
-  // not -- use the max times the unroll, and a floor so each block moves >= ~64 KB).
-  int rpb = max_rows_per_pass * kUnroll * 2;
-  if (rpb < 8) rpb = 8;
+  if (n_active == 0 || a.n == 0) return cudaSuccess;
+  // Rows per block: enough blocks for ~2 waves, each at least one unrolled pass.
+  const int per_rank_blocks = (kTargetBlocks + n_active * P - 1) / (n_active * P);
+  int rpb = (a.n + per_rank_blocks - 1) / per_rank_blocks;
+  const int unit = max_rows_per_pass * kUnroll;
+  rpb = (rpb + unit - 1) / unit * unit;
   a.rows_per_block = rpb;
-  dim3 grid((a.n + rpb - 1) / rpb, 3 * P);
+  dim3 grid((a.n + rpb - 1) / rpb, n_active * P);
   if (seq_to_head)
     permute_kernel<true><<<grid, kThreads, 0, stream>>>(a);
   else

@@ -54,6 +54,22 @@ ULY_DEV bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t kernel, uint32_t 
   report_error(kernel, site);
   return false;
 }
+// Bounded wait in warp-collective code (TMEM loads/stores, warp votes follow):
+// every lane polls, and the warp proceeds only if every lane saw the phase
+// complete, so a give-up never splits the warp.
+ULY_DEV bool mbar_wait_warp(uint32_t bar, uint32_t parity, uint32_t kernel, uint32_t site) {
+  const bool ok = mbar_wait(bar, parity, kernel, site);
+  return __all_sync(0xffffffffu, ok);
+}
+// Wait used when draining a CTA before exit (copies or MMAs it issued must land
+// before its shared memory and TMEM go away): always the built-in cap, never the
+// lowered test cap, so an early give-up elsewhere cannot cut the drain short.
+ULY_DEV bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint32_t kernel, uint32_t site) {
+  for (uint32_t i = 0; i < kDefaultWaitPolls; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  report_error(kernel, site);
+  return false;
+}
 
 // ---------------------------------------------------------------- TMA
 ULY_DEV void tma_prefetch_desc(const CUtensorMap* m) {

@@ -3,5 +3,5 @@
 #include <string.h>
 #include "permute.cu"
 #include "attn_fwd_sm100.cu"
-#include "attn_bwd_mma.cu"
+#include "attn_bwd_sm100.cu"
 #include "api.cu"

@@ -4,8 +4,8 @@ This module is shared by the CUDA path's tests/bench and by the CPU oracle.
 It holds NO arithmetic of the method itself: it only names the workload
 shapes, draws seeded random numbers, rounds them to bf16 once, and cuts the
 unsharded token axis into the P contiguous sequence shards the method starts
-from (each GPU "grabs its chunk of tokens, N/P" -- theaicatchup.com,
-"How Does Ulysses Sequence Parallelism Actually Work?").
+from (each rank first takes one contiguous N/P-token piece of the sequence --
+theaicatchup.com, "How Does Ulysses Sequence Parallelism Actually Work?").
 
 Recipe (one numpy ``Generator(PCG64(seed))`` stream per workload, drawn in
 this order): document lengths (packed-varlen workloads only), then Q, K, V,
