@@ -142,6 +142,33 @@ ULY_API uly_status ulysses_attn_bwd(
     void* workspace, size_t workspace_bytes,
     int rank_lo, int rank_hi, cudaStream_t stream);
 
+/* The attention backward for callers that cannot allocate device memory: a
+ * plugin or embedded runtime that hands this library only its input and output
+ * buffers and owns every allocation itself, or a loop where cudaMalloc (which
+ * can synchronise the device) is not allowed. The paper has no counterpart;
+ * this is a deployment variant of ulysses_attn_bwd with identical arguments
+ * and results, minus workspace/workspace_bytes.
+ *
+ * Its scratch is a fixed 32 MiB device array inside this library (held by every
+ * GPU that loads the library until the process exits); it needs
+ * ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d) <= 32 MiB, i.e.
+ * H * (N rounded up to a multiple of 128) <= 4,194,304 (for example
+ * N <= 131072 at H = 32); larger sizes return ULY_ERR_UNSUPPORTED with nothing
+ * launched. It calls no allocator. The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture. Every call shares the one
+ * array and leaves its contents behind; the kernels overwrite all of it that
+ * they read, so nothing needs clearing, but calls that overlap on the GPU (on
+ * different streams, or from different threads) race on it: serialise them. */
+ULY_API uly_status ulysses_attn_bwd_noalloc(
+    const void* const* q_head, const void* const* k_head, const void* const* v_head,
+    const void* const* o_head, const float* const* lse_head, const void* const* do_head,
+    void* const* dq_head, void* const* dk_head, void* const* dv_head,
+    int64_t N, int P, int H, int H_kv, int d,
+    const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
+    float softmax_scale,
+    int rank_lo, int rank_hi, cudaStream_t stream);
+
 /* Static text for a status code. */
 ULY_API const char* ulysses_status_string(uly_status s);
 

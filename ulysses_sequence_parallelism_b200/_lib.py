@@ -41,6 +41,8 @@ _SIGS = {
     "ulysses_get_device_status": [_v, ctypes.POINTER(ctypes.c_uint32)],
     "ulysses_set_wait_limit": [ctypes.c_uint32],
     "ulysses_selftest_bounded_wait": [_v],
+    "ulysses_attn_bwd_noalloc": [_vpp, _vpp, _vpp, _vpp, _fpp, _vpp, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _v, _i,
+                                 _i, ctypes.c_float, _i, _i, _v],
 }
 _RES = {"ulysses_attn_bwd_workspace_size": ctypes.c_size_t, "ulysses_status_string": ctypes.c_char_p,
         "ulysses_set_wait_limit": None}

@@ -5,3 +5,4 @@
 #include "attn_fwd_sm100.cu"
 #include "attn_bwd_sm100.cu"
 #include "api.cu"
+#include "bwd_noalloc.cu"
