@@ -99,6 +99,14 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def aggregate_over_ranks(local_ms: float, tokens_per_rank: int, world: int, reduce_max=None):
+    """Whole-job throughput for `world` ranks that each ran `tokens_per_rank`
+    tokens per step: the slowest rank's ms per step sets the job time. With a
+    process group, `reduce_max` is an all-reduce(max) over ranks."""
+    ms = reduce_max(local_ms) if (world > 1 and reduce_max is not None) else local_ms
+    return ms, world * tokens_per_rank / (ms / 1e3)
+
+
 def cpu_oracle_sample(w, inp, budget_s=20.0):
     """Time the fp64 oracle on a bounded sample of the workload and extrapolate
     the layer time linearly in (i, j) pairs x heads. Sample: forward + backward
@@ -290,12 +298,12 @@ def main():
     for s in range(args.steps):
         for i, st in enumerate(stages):
             stage_ms[st].append(evs[s][i].elapsed_time(evs[s][i + 1]))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
+    def reduce_max(x):
+        t = torch.tensor([x], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    ms_per_step = total_ms / args.steps
-    value = world * N / (ms_per_step / 1e3)
+        return float(t.item())
+
+    ms_per_step, value = aggregate_over_ranks(total_ms / args.steps, N, world, reduce_max)
 
     med = {st: statistics.median(v_) for st, v_ in stage_ms.items()}
     mean = {st: sum(v_) / len(v_) for st, v_ in stage_ms.items()}
@@ -358,12 +366,8 @@ def main():
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b) / args.steps
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * N / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e_ms, e_val = aggregate_over_ranks(a.elapsed_time(b) / args.steps, N, world, reduce_max)
+        e2e = {"value": e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
     cpu = None
