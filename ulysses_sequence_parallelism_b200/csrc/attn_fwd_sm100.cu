@@ -176,68 +176,88 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
+    // Order per key block j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1). S is issued
+    // as two N=64 halves; P lives in S's columns [0,64), so the upper half
+    // (columns 64..127) goes out right behind PV(j) and only the lower half
+    // waits for PV(j) to have read P -- the wait is hidden behind the upper half.
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
+      constexpr uint32_t idS = idesc_bf16_f32(BM, BN / 2, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(BM, D, 0, 1);
       bool ok = true;
 #pragma unroll
       for (int t = 0; t < 2; ++t)
         if (active[t] && !mbar_wait(q_full(t), 0, kErrFwd, 0x300 + t)) ok = false;
-      uint32_t it = 0;
+      auto part = [&](int t, int jb) { return active[t] && jb >= jb_begin[t] && jb < jb_end[t]; };
+      auto issue_s_half = [&](int t, uint32_t kb, int half) {
+        const uint32_t qb = sQ + t * L::kQTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(qb + (kk / 4) * (BM * 128) + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd =
+              smem_desc_sw128(kb + (kk / 4) * (BN * 128) + half * (64 * 128) + (kk % 4) * 32, 16, 1024);
+          mma_ss(tS[t] + half * 64, ad, bd, idS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, uint32_t vb, int cnt) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bd = smem_desc_sw128(vb + kk * (16 * 128), BN * 128, 1024);
+          mma_ts(tO[t], tS[t] + kk * 8, bd, idO, (cnt > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
       int cnt[2] = {0, 0};
-      for (int jb = jb_lo; jb < jb_hi && ok; ++jb) {
-        // K block -> S tiles
-        {
-          const int s = it % NSTAGE;
-          const uint32_t ph = (it / NSTAGE) & 1u;
-          ++it;
-          if (!mbar_wait(kv_full(s), ph, kErrFwd, 0x310)) { ok = false; break; }
+      // prologue: S for the first key block (ring slot 0)
+      if (ok && jb_lo < jb_hi) {
+        if (!mbar_wait(kv_full(0), 0, kErrFwd, 0x310)) {
+          ok = false;
+        } else {
           tc_fence_after();
-          const uint32_t kb = sRing + s * L::kKV;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
-            if (!active[t] || jb < jb_begin[t] || jb >= jb_end[t]) continue;
-            if (cnt[t] > 0) {
-              if (!mbar_wait(pv_done(t), (cnt[t] - 1) & 1, kErrFwd, 0x320 + t)) { ok = false; break; }
-              tc_fence_after();
-            }
-            const uint32_t qb = sQ + t * L::kQTile;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk / 4) * (BM * 128) + (kk % 4) * 32;
-              const uint64_t ad = smem_desc_sw128(qb + off, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(kb + (kk / 4) * (BN * 128) + (kk % 4) * 32, 16, 1024);
-              mma_ss(tS[t], ad, bd, idS, kk > 0 ? 1u : 0u);
-            }
+            if (!part(t, jb_lo)) continue;
+            issue_s_half(t, sRing, 1);
+            issue_s_half(t, sRing, 0);
             mma_commit(s_full(t));
           }
-          if (!ok) break;
-          mma_commit(kv_empty(s));
+          mma_commit(kv_empty(0));
         }
-        // V block -> O tiles
-        {
-          const int s = it % NSTAGE;
-          const uint32_t ph = (it / NSTAGE) & 1u;
-          ++it;
-          if (!mbar_wait(kv_full(s), ph, kErrFwd, 0x330)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t vb = sRing + s * L::kKV;
+      }
+      for (int jb = jb_lo; jb < jb_hi && ok; ++jb) {
+        const uint32_t itV = 2u * (jb - jb_lo) + 1u, itK = itV + 1u;
+        const bool has_next = jb + 1 < jb_hi;
+        if (!mbar_wait(kv_full(itV % NSTAGE), (itV / NSTAGE) & 1u, kErrFwd, 0x330)) { ok = false; break; }
+        if (has_next && !mbar_wait(kv_full(itK % NSTAGE), (itK / NSTAGE) & 1u, kErrFwd, 0x311)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t vb = sRing + (itV % NSTAGE) * L::kKV;
+        const uint32_t kb = sRing + (itK % NSTAGE) * L::kKV;
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (!active[t] || jb < jb_begin[t] || jb >= jb_end[t]) continue;
+        for (int t = 0; t < 2; ++t) {
+          const bool now = part(t, jb), nxt = has_next && part(t, jb + 1);
+          if (now) {
             if (!mbar_wait(p_full(t), cnt[t] & 1, kErrFwd, 0x340 + t)) { ok = false; break; }
             tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk) {
-              const uint64_t bd = smem_desc_sw128(vb + kk * (16 * 128), BN * 128, 1024);
-              mma_ts(tO[t], tS[t] + kk * 8, bd, idO, (cnt[t] > 0 || kk > 0) ? 1u : 0u);
-            }
+            issue_pv(t, vb, cnt[t]);
             mma_commit(pv_done(t));
+            if (nxt) {
+              issue_s_half(t, kb, 1);
+              if (!mbar_wait(pv_done(t), cnt[t] & 1, kErrFwd, 0x320 + t)) { ok = false; break; }
+              tc_fence_after();
+              issue_s_half(t, kb, 0);
+              mma_commit(s_full(t));
+            }
             ++cnt[t];
+          } else if (nxt) {
+            issue_s_half(t, kb, 1);
+            issue_s_half(t, kb, 0);
+            mma_commit(s_full(t));
           }
-          if (!ok) break;
-          mma_commit(kv_empty(s));
         }
+        if (!ok) break;
+        mma_commit(kv_empty(itV % NSTAGE));
+        if (has_next) mma_commit(kv_empty(itK % NSTAGE));
       }
       // Drain: wait for every MMA issued above before TMEM can be released.
       mma_commit(mma_done);
@@ -246,29 +266,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax / epilogue
+    // Per-warp scalars (no runtime-indexed arrays: they would live in local memory).
     const int t = warp >> 2;
     const int lrow = 32 * (warp & 3) + lane;        // TMEM lane = row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    if (active[t]) {
-      const int i = first_row[t] + lrow;
+    const int frow = m0 + t * BM;
+    const int lrow_t = min(frow + BM, N) - 1;
+    const uint32_t tSt = tmem + 128u * t, tOt = tmem + 256u + D * t;
+    if (frow < N) {
+      const int i = frow + lrow;
       const bool row_ok = i < N;
       const int st_i = doc_start_of(a.cu, a.num_seqs, min(i, N - 1));
-      const int max_start = doc_start_of(a.cu, a.num_seqs, last_row[t]);
+      const int max_start = doc_start_of(a.cu, a.num_seqs, lrow_t);
+      const int jbb = doc_start_of(a.cu, a.num_seqs, frow) / BN, jbe = lrow_t / BN + 1;
       const float sl2 = a.scale_log2;
       float m_run = -INFINITY, l_run = 0.f;
       int cnt = 0;
       bool ok = true;
-      for (int jb = jb_begin[t]; jb < jb_end[t]; ++jb, ++cnt) {
+      for (int jb = jbb; jb < jbe; ++jb, ++cnt) {
         if (!mbar_wait_warp(s_full(t), cnt & 1, kErrFwd, 0x400 + t)) { ok = false; break; }
         tc_fence_after();
         uint32_t v[BN];
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c)
-          tmem_ld32(tS[t] + lane_off + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
+          tmem_ld32(tSt + lane_off + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
         tmem_wait_ld();
         const int n0 = jb * BN;
-        const bool need_mask = (n0 + BN - 1 > first_row[t]) || (n0 < max_start);
-        float m_blk = -INFINITY;
+        const bool need_mask = (n0 + BN - 1 > frow) || (n0 < max_start);
+        float mx[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < BN; ++c) {
@@ -276,16 +303,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
             float x = u2f(v[c]) * sl2;
             x = (key > i || key < st_i) ? -INFINITY : x;
             v[c] = __float_as_uint(x);
-            m_blk = fmaxf(m_blk, x);
+            mx[c & 7] = fmaxf(mx[c & 7], x);
           }
         } else {
 #pragma unroll
           for (int c = 0; c < BN; ++c) {
             const float x = u2f(v[c]) * sl2;
             v[c] = __float_as_uint(x);
-            m_blk = fmaxf(m_blk, x);
+            mx[c & 7] = fmaxf(mx[c & 7], x);
           }
         }
+        const float m_blk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         const float m_new = fmaxf(m_run, m_blk);
         // Rescale decision (warp-uniform: TMEM loads/stores are warp-collective).
         bool rescale = false;
@@ -299,17 +328,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
           m_run = m_new;
         }
         const float base = (m_run == -INFINITY) ? 0.f : m_run;
-        float rs = 0.f;
+        float rs[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) rs[e] = 0.f;
 #pragma unroll
         for (int c = 0; c < BN; c += 2) {
           const float p0 = ex2_approx(u2f(v[c]) - base);
           const float p1 = ex2_approx(u2f(v[c + 1]) - base);
-          rs += p0 + p1;
+          rs[(c >> 1) & 7] += p0 + p1;
           v[c / 2] = pack_bf16x2(p0, p1);
         }
-        l_run += rs;
-        tmem_st32(tS[t] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_st32(tS[t] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        l_run += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+        tmem_st32(tSt + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_st32(tSt + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         if (rescale) {
           // O still holds the sum over earlier blocks at the old max: scale it
           // once the previous P.V has landed, before this block's P.V is issued.
@@ -318,11 +349,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
 #pragma unroll 1
           for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t ov[32];
-            tmem_ld32(tO[t] + lane_off + c4 * 32, ov);
+            tmem_ld32(tOt + lane_off + c4 * 32, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(u2f(ov[e]) * alpha);
-            tmem_st32(tO[t] + lane_off + c4 * 32, ov);
+            tmem_st32(tOt + lane_off + c4 * 32, ov);
           }
         }
         tmem_wait_st();
@@ -337,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
 #pragma unroll 1
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t ov[32];
-          tmem_ld32(tO[t] + lane_off + c4 * 32, ov);
+          tmem_ld32(tOt + lane_off + c4 * 32, ov);
           tmem_wait_ld();
           uint4 pk[4];
           uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
