@@ -25,3 +25,22 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(autouse=True, scope="session")
+def _short_device_wait_cap(request):
+    """GPU tests run with a shorter cap on bounded device waits (2^20 polls), so
+    that a kernel bug shows up as a prompt ULY_ERR_TIMEOUT instead of a long
+    stall; legitimate waits are microseconds."""
+    try:
+        import torch
+        if not torch.cuda.is_available():
+            yield
+            return
+        import ulysses_sequence_parallelism_b200 as U
+        U.ulysses_set_wait_limit(1 << 20)
+    except Exception:
+        yield
+        return
+    yield
+    U.ulysses_set_wait_limit(0)

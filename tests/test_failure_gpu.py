@@ -17,7 +17,7 @@ def test_bounded_wait_gives_up_and_reports():
         U.ulysses_selftest_bounded_wait()
         code, word = U.ulysses_get_device_status()
     finally:
-        U.ulysses_set_wait_limit(0)
+        U.ulysses_set_wait_limit(1 << 20)      # the session's test cap (see conftest)
     assert code == 4                       # ULY_ERR_TIMEOUT
     assert word == (0x7F << 24) | 0xABC    # kernel id, site
     assert U.ulysses_get_device_status() == (0, 0)   # read-and-clear

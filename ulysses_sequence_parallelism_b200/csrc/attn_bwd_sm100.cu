@@ -129,8 +129,9 @@ struct DkdvLayout {
   static constexpr uint32_t kRing = 2 * kKV;          // stage s: Q at +0, dO at +kBlk
   static constexpr uint32_t kVec = kRing + NST * 2 * kBlk;   // stage s: lse2 at +0, D at +256
   static constexpr uint32_t kBars = kVec + NST * 512;
-  // kv_full, st_full[NST], st_empty[NST], s_full[2], dp_full[2], p_full[2], ds_full[2], buf_free[2], acc_done
-  static constexpr int kNumBars = 1 + 2 * NST + 10 + 1;
+  // kv_full, st_full[NST], st_empty[NST], s_full[2], dp_full[2], p_full[2], ds_full[2], dv_done[2],
+  // dk_done[2], acc_done
+  static constexpr int kNumBars = 1 + 2 * NST + 12 + 1;
   static constexpr uint32_t kSlot = kBars + kNumBars * 8;
   static constexpr uint32_t kAlloc = kSlot + 16 + 1024;
 };
@@ -149,8 +150,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid
   auto dp_full = [&](int b) { return bars + 8u * (3 + 2 * NST + b); };
   auto p_full = [&](int b) { return bars + 8u * (5 + 2 * NST + b); };
   auto ds_full = [&](int b) { return bars + 8u * (7 + 2 * NST + b); };
-  auto buf_free = [&](int b) { return bars + 8u * (9 + 2 * NST + b); };
-  const uint32_t acc_done = bars + 8u * (11 + 2 * NST);
+  auto dv_done = [&](int b) { return bars + 8u * (9 + 2 * NST + b); };
+  auto dk_done = [&](int b) { return bars + 8u * (11 + 2 * NST + b); };
+  const uint32_t acc_done = bars + 8u * (13 + 2 * NST);
   volatile uint32_t* slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,94 +188,114 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid
   auto tDP = [&](int b) { return tmem + 256u + 128u * b + 64u; };
 
   if (warp == kTmaWarp) {
-    if (lane == 0) {
+    {
       const CUtensorMap *mq = &a.tq[r], *mdo = &a.tdo[r], *mk = &a.tk[r], *mv = &a.tv[r];
-      tma_prefetch_desc(mq);
-      tma_prefetch_desc(mdo);
-      mbar_arrive_expect_tx(kv_full, 2 * L::kKV);
+      if (lane == 0) tma_prefetch_desc(mq);
+      if (lane == 0) tma_prefetch_desc(mdo);
+      mbar_arrive_expect_tx_w(kv_full, 2 * L::kKV);
 #pragma unroll
       for (int hf = 0; hf < D / 64; ++hf) {
-        tma_load_2d(sbase + L::kK + hf * (TB * 128), mk, kv_full, g * D + hf * 64, n0);
-        tma_load_2d(sbase + L::kV + hf * (TB * 128), mv, kv_full, g * D + hf * 64, n0);
+        tma_load_2d_w(sbase + L::kK + hf * (TB * 128), mk, kv_full, g * D + hf * 64, n0);
+        tma_load_2d_w(sbase + L::kV + hf * (TB * 128), mv, kv_full, g * D + hf * 64, n0);
       }
       int it = 0;
       for (; it < T; ++it) {
         const int s = it % NST;
-        if (!mbar_wait(st_empty(s), ((it / NST) & 1) ^ 1, kErrBwd, 0x100 + s)) break;
+        if (!mbar_wait_warp(st_empty(s), ((it / NST) & 1) ^ 1, kErrBwd, 0x100 + s)) break;
         const int h = g * a.group + it / nrb;
         const int m0 = (rb_lo + it % nrb) * SB;
         const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
-        mbar_arrive_expect_tx(st_full(s), 2 * L::kBlk + 512);
+        mbar_arrive_expect_tx_w(st_full(s), 2 * L::kBlk + 512);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf) {
-          tma_load_2d(stg + hf * (SB * 128), mq, st_full(s), h * D + hf * 64, m0);
-          tma_load_2d(stg + L::kBlk + hf * (SB * 128), mdo, st_full(s), h * D + hf * 64, m0);
+          tma_load_2d_w(stg + hf * (SB * 128), mq, st_full(s), h * D + hf * 64, m0);
+          tma_load_2d_w(stg + L::kBlk + hf * (SB * 128), mdo, st_full(s), h * D + hf * 64, m0);
         }
         const int64_t vo = (static_cast<int64_t>(r) * a.Hl + h) * a.Npad + m0;
-        bulk_load(sbase + L::kVec + s * 512, a.lse2 + vo, SB * 4, st_full(s));
-        bulk_load(sbase + L::kVec + s * 512 + 256, a.Dv + vo, SB * 4, st_full(s));
+        bulk_load_w(sbase + L::kVec + s * 512, a.lse2 + vo, SB * 4, st_full(s));
+        bulk_load_w(sbase + L::kVec + s * 512 + 256, a.Dv + vo, SB * 4, st_full(s));
       }
       for (int k = it > NST ? it - NST : 0; k < it; ++k)
-        mbar_wait_drain(st_full(k % NST), (k / NST) & 1, kErrBwd, 0x1f0);
-      mbar_wait_drain(kv_full, 0, kErrBwd, 0x1f1);
+        mbar_wait_drain_w(st_full(k % NST), (k / NST) & 1, kErrBwd, 0x1f0);
+      mbar_wait_drain_w(kv_full, 0, kErrBwd, 0x1f1);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
+    {
+      // Tensor-pipe order: S^T(i+1) dP^T(i+1) | dV(i) dK(i) | S^T(i+2) dP^T(i+2) | ...
+      // S^T(i+2) reuses the columns dV(i) reads (P^T) and dP^T(i+2) the ones dK(i)
+      // reads (dS^T): each waits only for its own reader, so one is always queued.
       constexpr uint32_t idS = idesc_bf16_f32(TB, SB, 0, 0);
       constexpr uint32_t idA = idesc_bf16_f32(TB, D, 0, 1);
-      bool ok = mbar_wait(kv_full, 0, kErrBwd, 0x200);
+      bool ok = mbar_wait_warp(kv_full, 0, kErrBwd, 0x200);
       tc_fence_after();
-      auto issue_sdp = [&](int it) -> bool {
-        const int b = it & 1, s = it % NST;
-        if (!mbar_wait(st_full(s), (it / NST) & 1, kErrBwd, 0x210)) return false;
-        if (it >= 2 && !mbar_wait(buf_free(b), ((it - 2) >> 1) & 1, kErrBwd, 0x220)) return false;
-        tc_fence_after();
-        const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
+      auto stage = [&](int it) { return sbase + L::kRing + (it % NST) * 2 * L::kBlk; };
+      // Descriptors built once; per MMA only a constant offset is added.
+      const uint64_t dK0 = smem_desc_sw128(sbase + L::kK, 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(sbase + L::kV, 16, 1024);
+      const uint64_t dRing0 = smem_desc_sw128(sbase + L::kRing, 16, 1024);
+      const uint64_t dRingMN0 = smem_desc_sw128(sbase + L::kRing, SB * 128, 1024);
+      auto issue_s = [&](int it) {
+        const uint64_t qd = desc_adv(dRing0, (it % NST) * 2 * L::kBlk);
+        const uint32_t dst = tS(it & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk / 4) * (TB * 128) + (kk % 4) * 32;
           const uint32_t qo = (kk / 4) * (SB * 128) + (kk % 4) * 32;
-          mma_ss(tS(b), smem_desc_sw128(sbase + L::kK + ko, 16, 1024), smem_desc_sw128(stg + qo, 16, 1024), idS,
-                 kk > 0 ? 1u : 0u);
+          mma_ss_w(dst, desc_adv(dK0, ko), desc_adv(qd, qo), idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(s_full(b));
+        mma_commit_w(s_full(it & 1));
+      };
+      auto issue_dp = [&](int it) {
+        const uint64_t dod = desc_adv(dRing0, (it % NST) * 2 * L::kBlk + L::kBlk);
+        const uint32_t dst = tDP(it & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk / 4) * (TB * 128) + (kk % 4) * 32;
           const uint32_t qo = (kk / 4) * (SB * 128) + (kk % 4) * 32;
-          mma_ss(tDP(b), smem_desc_sw128(sbase + L::kV + ko, 16, 1024),
-                 smem_desc_sw128(stg + L::kBlk + qo, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          mma_ss_w(dst, desc_adv(dV0, ko), desc_adv(dod, qo), idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(dp_full(b));
-        return true;
+        mma_commit_w(dp_full(it & 1));
       };
-      auto issue_acc = [&](int it) -> bool {
-        const int b = it & 1, s = it % NST;
-        const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
-        if (!mbar_wait(p_full(b), (it >> 1) & 1, kErrBwd, 0x230)) return false;
+      // prologue: the first two streamed blocks
+      for (int it = 0; it < 2 && it < T && ok; ++it) {
+        if (!mbar_wait_warp(st_full(it % NST), (it / NST) & 1, kErrBwd, 0x210)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < SB / 16; ++kk)
-          mma_ts(tDV, tS(b) + kk * 8, smem_desc_sw128(stg + L::kBlk + kk * 2048, SB * 128, 1024), idA,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        if (!mbar_wait(ds_full(b), (it >> 1) & 1, kErrBwd, 0x240)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < SB / 16; ++kk)
-          mma_ts(tDK, tDP(b) + kk * 8, smem_desc_sw128(stg + kk * 2048, SB * 128, 1024), idA,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(st_empty(s));
-        mma_commit(buf_free(b));
-        return true;
-      };
-      if (ok && T > 0) ok = issue_sdp(0);
-      for (int it = 0; it < T && ok; ++it) {
-        if (it + 1 < T && !issue_sdp(it + 1)) { ok = false; break; }
-        ok = issue_acc(it);
+        issue_s(it);
+        issue_dp(it);
       }
-      mma_commit(acc_done);
-      mbar_wait_drain(acc_done, 0, kErrBwd, 0x250);
+      for (int it = 0; it < T && ok; ++it) {
+        const int b = it & 1;
+        const uint32_t stg = stage(it);
+        if (!mbar_wait_warp(p_full(b), (it >> 1) & 1, kErrBwd, 0x230)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t dob = desc_adv(dRingMN0, stg - (sbase + L::kRing) + L::kBlk);
+        const uint64_t qb = desc_adv(dRingMN0, stg - (sbase + L::kRing));
+        const uint32_t aS = tS(b), aDP = tDP(b);
+#pragma unroll
+        for (int kk = 0; kk < SB / 16; ++kk)
+          mma_ts_w(tDV, aS + kk * 8, desc_adv(dob, kk * 2048), idA, (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_w(dv_done(b));
+        if (!mbar_wait_warp(ds_full(b), (it >> 1) & 1, kErrBwd, 0x240)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < SB / 16; ++kk)
+          mma_ts_w(tDK, aDP + kk * 8, desc_adv(qb, kk * 2048), idA, (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_w(dk_done(b));
+        mma_commit_w(st_empty(it % NST));
+        const int nx = it + 2;
+        if (nx < T) {
+          if (!mbar_wait_warp(st_full(nx % NST), (nx / NST) & 1, kErrBwd, 0x210)) { ok = false; break; }
+          if (!mbar_wait_warp(dv_done(b), (it >> 1) & 1, kErrBwd, 0x220)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(nx);
+          if (!mbar_wait_warp(dk_done(b), (it >> 1) & 1, kErrBwd, 0x221)) { ok = false; break; }
+          tc_fence_after();
+          issue_dp(nx);
+        }
+      }
+      mma_commit_w(acc_done);
+      mbar_wait_drain_w(acc_done, 0, kErrBwd, 0x250);
     }
     __syncwarp();
   } else {
@@ -314,20 +336,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid
       mbar_arrive(p_full(b));
       if (!mbar_wait_warp(dp_full(b), (it >> 1) & 1, kErrBwd, 0x320)) { ok = false; break; }
       tc_fence_after();
+      uint32_t dp[SB];
+      tmem_ld32(tDP(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+      tmem_ld32(tDP(b) + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      tmem_wait_ld();
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t dp[32];
-        tmem_ld32(tDP(b) + loff + half * 32, dp);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int c0 = half * 32 + 2 * c;
-          const float d0 = u2f(pv[c0]) * (u2f(dp[2 * c]) - vd[c0]);
-          const float d1 = u2f(pv[c0 + 1]) * (u2f(dp[2 * c + 1]) - vd[c0 + 1]);
-          pk[half * 16 + c] = pack_bf16x2(d0, d1);
-        }
+      for (int c = 0; c < SB; c += 2) {
+        const float d0 = u2f(pv[c]) * (u2f(dp[c]) - vd[c]);
+        const float d1 = u2f(pv[c + 1]) * (u2f(dp[c + 1]) - vd[c + 1]);
+        dp[c / 2] = pack_bf16x2(d0, d1);     // in place: dp[c/2] is already consumed
       }
-      tmem_st32(tDP(b) + loff, pk);
+      tmem_st32(tDP(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(ds_full(b));
@@ -389,7 +408,7 @@ struct DqLayout {
   static constexpr uint32_t kQ = 0, kDO = kTile;
   static constexpr uint32_t kRing = 2 * kTile;        // stage s: K at +0, V at +kBlk
   static constexpr uint32_t kBars = kRing + NST * 2 * kBlk;
-  // q_full, st_full[NST], st_empty[NST], s_full[2], dp_full[2], ds_full[2], buf_free[2], acc_done
+  // q_full, st_full[NST], st_empty[NST], s_full[2], dp_full[2], ds_full[2], dq_done[2], acc_done
   static constexpr int kNumBars = 1 + 2 * NST + 8 + 1;
   static constexpr uint32_t kSlot = kBars + kNumBars * 8;
   static constexpr uint32_t kAlloc = kSlot + 16 + 1024;
@@ -408,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
   auto s_full = [&](int b) { return bars + 8u * (1 + 2 * NST + b); };
   auto dp_full = [&](int b) { return bars + 8u * (3 + 2 * NST + b); };
   auto ds_full = [&](int b) { return bars + 8u * (5 + 2 * NST + b); };
-  auto buf_free = [&](int b) { return bars + 8u * (7 + 2 * NST + b); };
+  auto dq_done = [&](int b) { return bars + 8u * (7 + 2 * NST + b); };
   const uint32_t acc_done = bars + 8u * (9 + 2 * NST);
   volatile uint32_t* slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kSlot);
 
@@ -442,84 +461,101 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
   auto tDP = [&](int b) { return tmem + 128u + 128u * b + 64u; };
 
   if (warp == kTmaWarp) {
-    if (lane == 0) {
+    {
       const CUtensorMap *mq = &a.tq[r], *mdo = &a.tdo[r], *mk = &a.tk[r], *mv = &a.tv[r];
-      tma_prefetch_desc(mk);
-      tma_prefetch_desc(mv);
-      mbar_arrive_expect_tx(q_full, 2 * L::kTile);
+      if (lane == 0) tma_prefetch_desc(mk);
+      if (lane == 0) tma_prefetch_desc(mv);
+      mbar_arrive_expect_tx_w(q_full, 2 * L::kTile);
 #pragma unroll
       for (int hf = 0; hf < D / 64; ++hf) {
-        tma_load_2d(sbase + L::kQ + hf * (TB * 128), mq, q_full, h * D + hf * 64, m0);
-        tma_load_2d(sbase + L::kDO + hf * (TB * 128), mdo, q_full, h * D + hf * 64, m0);
+        tma_load_2d_w(sbase + L::kQ + hf * (TB * 128), mq, q_full, h * D + hf * 64, m0);
+        tma_load_2d_w(sbase + L::kDO + hf * (TB * 128), mdo, q_full, h * D + hf * 64, m0);
       }
       int it = 0;
       for (; it < T; ++it) {
         const int s = it % NST;
-        if (!mbar_wait(st_empty(s), ((it / NST) & 1) ^ 1, kErrBwd, 0x500 + s)) break;
+        if (!mbar_wait_warp(st_empty(s), ((it / NST) & 1) ^ 1, kErrBwd, 0x500 + s)) break;
         const int k0 = (kb_lo + it) * SB;
         const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
-        mbar_arrive_expect_tx(st_full(s), 2 * L::kBlk);
+        mbar_arrive_expect_tx_w(st_full(s), 2 * L::kBlk);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf) {
-          tma_load_2d(stg + hf * (SB * 128), mk, st_full(s), g * D + hf * 64, k0);
-          tma_load_2d(stg + L::kBlk + hf * (SB * 128), mv, st_full(s), g * D + hf * 64, k0);
+          tma_load_2d_w(stg + hf * (SB * 128), mk, st_full(s), g * D + hf * 64, k0);
+          tma_load_2d_w(stg + L::kBlk + hf * (SB * 128), mv, st_full(s), g * D + hf * 64, k0);
         }
       }
       for (int k = it > NST ? it - NST : 0; k < it; ++k)
-        mbar_wait_drain(st_full(k % NST), (k / NST) & 1, kErrBwd, 0x5f0);
-      mbar_wait_drain(q_full, 0, kErrBwd, 0x5f1);
+        mbar_wait_drain_w(st_full(k % NST), (k / NST) & 1, kErrBwd, 0x5f0);
+      mbar_wait_drain_w(q_full, 0, kErrBwd, 0x5f1);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
+    {
+      // Tensor-pipe order: S(i+1) dP(i+1) | dQ(i) | dP(i+2) S(i+2) | dQ(i+1) ...
+      // dP(i+2) does not touch the columns dQ(i) reads (dS sits over S), so it
+      // is issued at once; only S(i+2) waits for dQ(i) to have read dS.
       constexpr uint32_t idS = idesc_bf16_f32(TB, SB, 0, 0);
       constexpr uint32_t idA = idesc_bf16_f32(TB, D, 0, 1);
-      bool ok = mbar_wait(q_full, 0, kErrBwd, 0x600);
+      bool ok = mbar_wait_warp(q_full, 0, kErrBwd, 0x600);
       tc_fence_after();
-      auto issue_sdp = [&](int it) -> bool {
-        const int b = it & 1, s = it % NST;
-        if (!mbar_wait(st_full(s), (it / NST) & 1, kErrBwd, 0x610)) return false;
-        if (it >= 2 && !mbar_wait(buf_free(b), ((it - 2) >> 1) & 1, kErrBwd, 0x620)) return false;
-        tc_fence_after();
-        const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
+      auto stage = [&](int it) { return sbase + L::kRing + (it % NST) * 2 * L::kBlk; };
+      // Descriptors built once; per MMA only a constant offset is added.
+      const uint64_t dQ0 = smem_desc_sw128(sbase + L::kQ, 16, 1024);
+      const uint64_t dDO0 = smem_desc_sw128(sbase + L::kDO, 16, 1024);
+      const uint64_t dRing0 = smem_desc_sw128(sbase + L::kRing, 16, 1024);
+      const uint64_t dRingMN0 = smem_desc_sw128(sbase + L::kRing, SB * 128, 1024);
+      auto issue_s = [&](int it) {
+        const uint64_t kd = desc_adv(dRing0, (it % NST) * 2 * L::kBlk);
+        const uint32_t dst = tS(it & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qo = (kk / 4) * (TB * 128) + (kk % 4) * 32;
           const uint32_t ko = (kk / 4) * (SB * 128) + (kk % 4) * 32;
-          mma_ss(tS(b), smem_desc_sw128(sbase + L::kQ + qo, 16, 1024), smem_desc_sw128(stg + ko, 16, 1024), idS,
-                 kk > 0 ? 1u : 0u);
+          mma_ss_w(dst, desc_adv(dQ0, qo), desc_adv(kd, ko), idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(s_full(b));
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qo = (kk / 4) * (TB * 128) + (kk % 4) * 32;
-          const uint32_t ko = (kk / 4) * (SB * 128) + (kk % 4) * 32;
-          mma_ss(tDP(b), smem_desc_sw128(sbase + L::kDO + qo, 16, 1024),
-                 smem_desc_sw128(stg + L::kBlk + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(dp_full(b));
-        return true;
+        mma_commit_w(s_full(it & 1));
       };
-      auto issue_acc = [&](int it) -> bool {
-        const int b = it & 1, s = it % NST;
-        const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
-        if (!mbar_wait(ds_full(b), (it >> 1) & 1, kErrBwd, 0x630)) return false;
+      auto issue_dp = [&](int it) {
+        const uint64_t vd = desc_adv(dRing0, (it % NST) * 2 * L::kBlk + L::kBlk);
+        const uint32_t dst = tDP(it & 1);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qo = (kk / 4) * (TB * 128) + (kk % 4) * 32;
+          const uint32_t ko = (kk / 4) * (SB * 128) + (kk % 4) * 32;
+          mma_ss_w(dst, desc_adv(dDO0, qo), desc_adv(vd, ko), idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit_w(dp_full(it & 1));
+      };
+      for (int it = 0; it < 2 && it < T && ok; ++it) {
+        if (!mbar_wait_warp(st_full(it % NST), (it / NST) & 1, kErrBwd, 0x610)) { ok = false; break; }
         tc_fence_after();
+        issue_s(it);
+        issue_dp(it);
+      }
+      for (int it = 0; it < T && ok; ++it) {
+        const int b = it & 1;
+        const uint32_t stg = stage(it);
+        if (!mbar_wait_warp(ds_full(b), (it >> 1) & 1, kErrBwd, 0x630)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t kb = desc_adv(dRingMN0, stg - (sbase + L::kRing));
+        const uint32_t aS = tS(b);
 #pragma unroll
         for (int kk = 0; kk < SB / 16; ++kk)
-          mma_ts(tDQ, tS(b) + kk * 8, smem_desc_sw128(stg + kk * 2048, SB * 128, 1024), idA,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(st_empty(s));
-        mma_commit(buf_free(b));
-        return true;
-      };
-      if (ok && T > 0) ok = issue_sdp(0);
-      for (int it = 0; it < T && ok; ++it) {
-        if (it + 1 < T && !issue_sdp(it + 1)) { ok = false; break; }
-        ok = issue_acc(it);
+          mma_ts_w(tDQ, aS + kk * 8, desc_adv(kb, kk * 2048), idA, (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_w(dq_done(b));
+        mma_commit_w(st_empty(it % NST));
+        const int nx = it + 2;
+        if (nx < T) {
+          if (!mbar_wait_warp(st_full(nx % NST), (nx / NST) & 1, kErrBwd, 0x610)) { ok = false; break; }
+          tc_fence_after();
+          issue_dp(nx);
+          if (!mbar_wait_warp(dq_done(b), (it >> 1) & 1, kErrBwd, 0x620)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(nx);
+        }
       }
-      mma_commit(acc_done);
-      mbar_wait_drain(acc_done, 0, kErrBwd, 0x640);
+      mma_commit_w(acc_done);
+      mbar_wait_drain_w(acc_done, 0, kErrBwd, 0x640);
     }
     __syncwarp();
   } else {
@@ -539,34 +575,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
       const int k0 = (kb_lo + it) * SB;
       if (!mbar_wait_warp(s_full(b), (it >> 1) & 1, kErrBwd, 0x700)) { ok = false; break; }
       tc_fence_after();
-      uint32_t pv[SB];
+      uint32_t pv[SB], dp[SB];
       tmem_ld32(tS(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
       tmem_ld32(tS(b) + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
+      if (!mbar_wait_warp(dp_full(b), (it >> 1) & 1, kErrBwd, 0x710)) { ok = false; break; }
+      tc_fence_after();
+      tmem_ld32(tDP(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+      tmem_ld32(tDP(b) + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
       tmem_wait_ld();
       const bool need_mask = (k0 + SB - 1 > m0) || (k0 < max_start);
 #pragma unroll
-      for (int c = 0; c < SB; ++c) {
-        const int key = k0 + c;
-        float p = ex2_approx(u2f(pv[c]) * sl2 - lse2_i);
-        if (need_mask && (key > i || key < st_i)) p = 0.f;
-        pv[c] = __float_as_uint(p);
-      }
-      if (!mbar_wait_warp(dp_full(b), (it >> 1) & 1, kErrBwd, 0x710)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t pk[SB / 2];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t dp[32];
-        tmem_ld32(tDP(b) + loff + half * 32, dp);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int c0 = half * 32 + 2 * c;
-          pk[half * 16 + c] = pack_bf16x2(u2f(pv[c0]) * (u2f(dp[2 * c]) - D_i),
-                                          u2f(pv[c0 + 1]) * (u2f(dp[2 * c + 1]) - D_i));
+      for (int c = 0; c < SB; c += 2) {
+        float p0 = ex2_approx(u2f(pv[c]) * sl2 - lse2_i);
+        float p1 = ex2_approx(u2f(pv[c + 1]) * sl2 - lse2_i);
+        if (need_mask) {
+          const int key = k0 + c;
+          if (key > i || key < st_i) p0 = 0.f;
+          if (key + 1 > i || key + 1 < st_i) p1 = 0.f;
         }
+        pv[c / 2] = pack_bf16x2(p0 * (u2f(dp[c]) - D_i), p1 * (u2f(dp[c + 1]) - D_i));   // in place
       }
-      tmem_st32(tS(b) + loff, pk);
+      tmem_st32(tS(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(ds_full(b));

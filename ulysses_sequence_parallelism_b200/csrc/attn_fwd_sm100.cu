@@ -135,20 +135,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    {
       const CUtensorMap* mq = &a.tq[r];
       const CUtensorMap* mk = &a.tk[r];
       const CUtensorMap* mv = &a.tv[r];
-      tma_prefetch_desc(mq);
-      tma_prefetch_desc(mk);
-      tma_prefetch_desc(mv);
+      if (lane == 0) tma_prefetch_desc(mq);
+      if (lane == 0) tma_prefetch_desc(mk);
+      if (lane == 0) tma_prefetch_desc(mv);
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (!active[t]) continue;
-        mbar_arrive_expect_tx(q_full(t), L::kQTile);
+        mbar_arrive_expect_tx_w(q_full(t), L::kQTile);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf)
-          tma_load_2d(sQ + t * L::kQTile + hf * (BM * 128), mq, q_full(t), h * D + hf * 64, first_row[t]);
+          tma_load_2d_w(sQ + t * L::kQTile + hf * (BM * 128), mq, q_full(t), h * D + hf * 64, first_row[t]);
       }
       uint32_t it = 0;
       bool ok = true;
@@ -157,21 +157,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
         for (int kind = 0; kind < 2; ++kind, ++it) {
           const int s = it % NSTAGE;
           const uint32_t ph = (it / NSTAGE) & 1u;
-          if (!mbar_wait(kv_empty(s), ph ^ 1u, kErrFwd, 0x100 + s)) { ok = false; break; }
-          mbar_arrive_expect_tx(kv_full(s), L::kKV);
+          if (!mbar_wait_warp(kv_empty(s), ph ^ 1u, kErrFwd, 0x100 + s)) { ok = false; break; }
+          mbar_arrive_expect_tx_w(kv_full(s), L::kKV);
           const CUtensorMap* m = kind == 0 ? mk : mv;
 #pragma unroll
           for (int hf = 0; hf < D / 64; ++hf)
-            tma_load_2d(sRing + s * L::kKV + hf * (BN * 128), m, kv_full(s), g * D + hf * 64, jb * BN);
+            tma_load_2d_w(sRing + s * L::kKV + hf * (BN * 128), m, kv_full(s), g * D + hf * 64, jb * BN);
         }
       }
       // Drain: every issued load must land before the CTA can exit.
       const uint32_t issued = it;
       for (uint32_t k = issued > NSTAGE ? issued - NSTAGE : 0; k < issued; ++k)
-        mbar_wait_drain(kv_full(k % NSTAGE), (k / NSTAGE) & 1u, kErrFwd, 0x200);
+        mbar_wait_drain_w(kv_full(k % NSTAGE), (k / NSTAGE) & 1u, kErrFwd, 0x200);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-        if (active[t]) mbar_wait_drain(q_full(t), 0, kErrFwd, 0x210 + t);
+        if (active[t]) mbar_wait_drain_w(q_full(t), 0, kErrFwd, 0x210 + t);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -180,35 +180,40 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
     // as two N=64 halves; P lives in S's columns [0,64), so the upper half
     // (columns 64..127) goes out right behind PV(j) and only the lower half
     // waits for PV(j) to have read P -- the wait is hidden behind the upper half.
-    if (lane == 0) {
+    {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN / 2, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(BM, D, 0, 1);
       bool ok = true;
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-        if (active[t] && !mbar_wait(q_full(t), 0, kErrFwd, 0x300 + t)) ok = false;
+        if (active[t] && !mbar_wait_warp(q_full(t), 0, kErrFwd, 0x300 + t)) ok = false;
       auto part = [&](int t, int jb) { return active[t] && jb >= jb_begin[t] && jb < jb_end[t]; };
+      // Descriptors built once; per MMA only a constant offset is added.
+      const uint64_t dQ0 = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dRing0 = smem_desc_sw128(sRing, 16, 1024);
+      const uint64_t dRingV0 = smem_desc_sw128(sRing, BN * 128, 1024);
       auto issue_s_half = [&](int t, uint32_t kb, int half) {
-        const uint32_t qb = sQ + t * L::kQTile;
+        const uint64_t qd = desc_adv(dQ0, t * L::kQTile);
+        const uint64_t kd = desc_adv(dRing0, kb - sRing + half * (64 * 128));
+        const uint32_t dst = tS[t] + half * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(qb + (kk / 4) * (BM * 128) + (kk % 4) * 32, 16, 1024);
-          const uint64_t bd =
-              smem_desc_sw128(kb + (kk / 4) * (BN * 128) + half * (64 * 128) + (kk % 4) * 32, 16, 1024);
-          mma_ss(tS[t] + half * 64, ad, bd, idS, kk > 0 ? 1u : 0u);
+          const uint32_t off_q = (kk / 4) * (BM * 128) + (kk % 4) * 32;
+          const uint32_t off_k = (kk / 4) * (BN * 128) + (kk % 4) * 32;
+          mma_ss_w(dst, desc_adv(qd, off_q), desc_adv(kd, off_k), idS, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, uint32_t vb, int cnt) {
+        const uint64_t vd = desc_adv(dRingV0, vb - sRing);
+        const uint32_t a0 = tS[t], dst = tO[t];
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(vb + kk * (16 * 128), BN * 128, 1024);
-          mma_ts(tO[t], tS[t] + kk * 8, bd, idO, (cnt > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts_w(dst, a0 + kk * 8, desc_adv(vd, kk * (16 * 128)), idO, (cnt > 0 || kk > 0) ? 1u : 0u);
       };
       int cnt[2] = {0, 0};
       // prologue: S for the first key block (ring slot 0)
       if (ok && jb_lo < jb_hi) {
-        if (!mbar_wait(kv_full(0), 0, kErrFwd, 0x310)) {
+        if (!mbar_wait_warp(kv_full(0), 0, kErrFwd, 0x310)) {
           ok = false;
         } else {
           tc_fence_after();
@@ -217,16 +222,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
             if (!part(t, jb_lo)) continue;
             issue_s_half(t, sRing, 1);
             issue_s_half(t, sRing, 0);
-            mma_commit(s_full(t));
+            mma_commit_w(s_full(t));
           }
-          mma_commit(kv_empty(0));
+          mma_commit_w(kv_empty(0));
         }
       }
       for (int jb = jb_lo; jb < jb_hi && ok; ++jb) {
         const uint32_t itV = 2u * (jb - jb_lo) + 1u, itK = itV + 1u;
         const bool has_next = jb + 1 < jb_hi;
-        if (!mbar_wait(kv_full(itV % NSTAGE), (itV / NSTAGE) & 1u, kErrFwd, 0x330)) { ok = false; break; }
-        if (has_next && !mbar_wait(kv_full(itK % NSTAGE), (itK / NSTAGE) & 1u, kErrFwd, 0x311)) {
+        if (!mbar_wait_warp(kv_full(itV % NSTAGE), (itV / NSTAGE) & 1u, kErrFwd, 0x330)) { ok = false; break; }
+        if (has_next && !mbar_wait_warp(kv_full(itK % NSTAGE), (itK / NSTAGE) & 1u, kErrFwd, 0x311)) {
           ok = false;
           break;
         }
@@ -237,31 +242,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
         for (int t = 0; t < 2; ++t) {
           const bool now = part(t, jb), nxt = has_next && part(t, jb + 1);
           if (now) {
-            if (!mbar_wait(p_full(t), cnt[t] & 1, kErrFwd, 0x340 + t)) { ok = false; break; }
+            if (!mbar_wait_warp(p_full(t), cnt[t] & 1, kErrFwd, 0x340 + t)) { ok = false; break; }
             tc_fence_after();
             issue_pv(t, vb, cnt[t]);
-            mma_commit(pv_done(t));
+            mma_commit_w(pv_done(t));
             if (nxt) {
               issue_s_half(t, kb, 1);
-              if (!mbar_wait(pv_done(t), cnt[t] & 1, kErrFwd, 0x320 + t)) { ok = false; break; }
+              if (!mbar_wait_warp(pv_done(t), cnt[t] & 1, kErrFwd, 0x320 + t)) { ok = false; break; }
               tc_fence_after();
               issue_s_half(t, kb, 0);
-              mma_commit(s_full(t));
+              mma_commit_w(s_full(t));
             }
             ++cnt[t];
           } else if (nxt) {
             issue_s_half(t, kb, 1);
             issue_s_half(t, kb, 0);
-            mma_commit(s_full(t));
+            mma_commit_w(s_full(t));
           }
         }
         if (!ok) break;
-        mma_commit(kv_empty(itV % NSTAGE));
-        if (has_next) mma_commit(kv_empty(itK % NSTAGE));
+        mma_commit_w(kv_empty(itV % NSTAGE));
+        if (has_next) mma_commit_w(kv_empty(itK % NSTAGE));
       }
       // Drain: wait for every MMA issued above before TMEM can be released.
-      mma_commit(mma_done);
-      mbar_wait_drain(mma_done, 0, kErrFwd, 0x350);
+      mma_commit_w(mma_done);
+      mbar_wait_drain_w(mma_done, 0, kErrFwd, 0x350);
     }
     __syncwarp();
   } else {

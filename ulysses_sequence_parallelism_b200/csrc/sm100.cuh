@@ -150,6 +150,59 @@ ULY_DEV void tmem_st16(uint32_t taddr, const uint32_t* r) {
 ULY_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 ULY_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ---------------------------------------------------------------- warp-converged issue
+// The variants below are executed by a whole converged warp; `elect.sync`
+// picks one lane to issue the instruction. Keeping the warp converged lets
+// the compiler hold descriptors and addresses in uniform registers, which is
+// what keeps a single issuing thread from becoming the bottleneck.
+ULY_DEV void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+ULY_DEV void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+ULY_DEV void mma_commit_w(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+ULY_DEV void mbar_arrive_expect_tx_w(uint32_t bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b64 st;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+      "r"(bytes)
+      : "memory");
+}
+ULY_DEV void tma_load_2d_w(uint32_t dst, const CUtensorMap* m, uint32_t bar, int x, int y) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+      "\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+ULY_DEV void bulk_load_w(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// Warp-converged drain wait (every lane polls; result made warp-uniform).
+ULY_DEV bool mbar_wait_drain_w(uint32_t bar, uint32_t parity, uint32_t kernel, uint32_t site) {
+  const bool ok = mbar_wait_drain(bar, parity, kernel, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor (sm_100 format): start address >> 4 in bits
 // [0,14), leading byte offset >> 4 in [16,30), stride byte offset >> 4 in
@@ -163,6 +216,13 @@ ULY_DEV uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sb
   d |= 2ull << 61;
   return d;
 }
+
+// Advance a descriptor's start address by a byte offset (a multiple of 16).
+// The start-address field holds address >> 4 in its low 14 bits; shared-memory
+// addresses stay below 2^18, so the add never carries out of the field. With a
+// compile-time offset this is one add: descriptors are built once per operand
+// and advanced per MMA, keeping the single issuing thread's chain short.
+ULY_DEV uint64_t desc_adv(uint64_t d, uint32_t byte_off) { return d + static_cast<uint64_t>(byte_off >> 4); }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
 // c_format bits [4,6) = 1 (F32); a_format [7,10) = 1 (BF16); b_format [10,13) = 1;
