@@ -19,14 +19,14 @@
 //              P^T, dS^T elementwise (one thread per key row), bf16 into TMEM
 //              dV += P^T dO,  dK += dS^T Q         (TS MMAs into TMEM)
 //  3. dq   : one CTA per 128-row block of one query head. Q and dO stay in
-//            shared memory; the CTA streams 64-key blocks of K and V:
-//              S = Q K^T, dP = dO V^T; dS elementwise (one thread per row);
-//              dQ += dS K (TS MMA into TMEM).
+//            shared memory; the CTA streams 128-key blocks of K and V:
+//              S = Q K^T, dP = dO V^T; dS elementwise (one thread per row,
+//              the two warpgroups on the two key halves); dQ += dS K (TS MMA).
 // S and dP are recomputed in (3): 7 block GEMMs instead of 5, in exchange for
 // no fp32 atomics, no dQ accumulator traffic and a bit-reproducible result.
-// Warp roles in 2 and 3: warps 0-3 / 4-7 elementwise (ping-pong on the two
-// TMEM buffers), warp 8 TMA producer, warp 9 MMA issuer. Every mbarrier wait
-// is bounded and reports into the library error word.
+// Warp roles in 2 and 3: warps 0-3 / 4-7 elementwise, warp 8 TMA producer,
+// warp 9 MMA issuer (TMA and MMA warps run converged; one elected lane issues).
+// Every mbarrier wait is bounded and reports into the library error word.
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -385,11 +385,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid
 }
 
 // ====================================================================== dQ
+// One CTA per 128-row block of one query head. Q and dO stay in shared memory;
+// 128-key blocks of K and V stream through two rings (K: 3 stages, V: 2), so
+// every MMA is N=128 wide (half the shared-memory operand traffic per FLOP of
+// 64-key blocks):
+//   S = Q K^T (S double-buffered in TMEM), dP = dO V^T (single buffer),
+//   dS = P (dP - D_i) elementwise: both warpgroups work on the same block, one
+//   thread per row, warpgroup w on keys [64w, 64w+64); each writes its dS as
+//   bf16 over the start of its own S columns, and dQ += dS K is issued as two
+//   K=64 halves that read those two column ranges.
+// Tensor-pipe order per block i: dP(i+1) | dQ(i) | S(i+2): dP(i+1) goes out as
+// soon as the elementwise warps have read dP(i), so they can start block i+1
+// while dQ(i) runs.
 struct DqArgs {
   CUtensorMap tq[kMaxRanks];    // box 64 cols x TB rows
   CUtensorMap tdo[kMaxRanks];   // box 64 cols x TB rows
-  CUtensorMap tk[kMaxRanks];    // box 64 cols x SB rows
-  CUtensorMap tv[kMaxRanks];    // box 64 cols x SB rows
+  CUtensorMap tk[kMaxRanks];    // box 64 cols x TB rows
+  CUtensorMap tv[kMaxRanks];    // box 64 cols x TB rows
   RankPtrsMut dq;
   const float* lse2;
   const float* Dv;
@@ -401,15 +413,17 @@ struct DqArgs {
   int num_m_tiles;
 };
 
+constexpr int kNK = 3, kNV = 2;   // K and V ring depths in the dQ kernel
+
 template <int D>
 struct DqLayout {
-  static constexpr uint32_t kTile = TB * D * 2;
-  static constexpr uint32_t kBlk = SB * D * 2;
+  static constexpr uint32_t kTile = TB * D * 2;        // 128 rows (or keys) x D
   static constexpr uint32_t kQ = 0, kDO = kTile;
-  static constexpr uint32_t kRing = 2 * kTile;        // stage s: K at +0, V at +kBlk
-  static constexpr uint32_t kBars = kRing + NST * 2 * kBlk;
-  // q_full, st_full[NST], st_empty[NST], s_full[2], dp_full[2], ds_full[2], dq_done[2], acc_done
-  static constexpr int kNumBars = 1 + 2 * NST + 8 + 1;
+  static constexpr uint32_t kKRing = 2 * kTile;
+  static constexpr uint32_t kVRing = kKRing + kNK * kTile;
+  static constexpr uint32_t kBars = kVRing + kNV * kTile;
+  // q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full[2], dp_full, ds_full, dq_done[2], acc_done
+  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 1 + 1 + 2 + 1;
   static constexpr uint32_t kSlot = kBars + kNumBars * 8;
   static constexpr uint32_t kAlloc = kSlot + 16 + 1024;
 };
@@ -422,13 +436,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
   const uint32_t bars = sbase + L::kBars;
   const uint32_t q_full = bars;
-  auto st_full = [&](int s) { return bars + 8u * (1 + s); };
-  auto st_empty = [&](int s) { return bars + 8u * (1 + NST + s); };
-  auto s_full = [&](int b) { return bars + 8u * (1 + 2 * NST + b); };
-  auto dp_full = [&](int b) { return bars + 8u * (3 + 2 * NST + b); };
-  auto ds_full = [&](int b) { return bars + 8u * (5 + 2 * NST + b); };
-  auto dq_done = [&](int b) { return bars + 8u * (7 + 2 * NST + b); };
-  const uint32_t acc_done = bars + 8u * (9 + 2 * NST);
+  auto k_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto k_empty = [&](int s) { return bars + 8u * (1 + kNK + s); };
+  auto v_full = [&](int s) { return bars + 8u * (1 + 2 * kNK + s); };
+  auto v_empty = [&](int s) { return bars + 8u * (1 + 2 * kNK + kNV + s); };
+  auto s_full = [&](int b) { return bars + 8u * (1 + 2 * kNK + 2 * kNV + b); };
+  const uint32_t dp_full = bars + 8u * (3 + 2 * kNK + 2 * kNV);
+  const uint32_t ds_full = bars + 8u * (4 + 2 * kNK + 2 * kNV);
+  auto dq_done = [&](int b) { return bars + 8u * (5 + 2 * kNK + 2 * kNV + b); };
+  const uint32_t acc_done = bars + 8u * (7 + 2 * kNK + 2 * kNV);
   volatile uint32_t* slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -438,14 +454,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
   const int N = a.N;
   const int m0 = (a.num_m_tiles - 1 - static_cast<int>(blockIdx.y)) * TB;   // longest first
   const int m_last = min(m0 + TB, N) - 1;
-  const int kb_lo = doc_start_of(a.cu, a.num_seqs, m0) / SB;
-  const int T = m_last / SB + 1 - kb_lo;
+  const int kb_lo = doc_start_of(a.cu, a.num_seqs, m0) / TB;
+  const int T = m_last / TB + 1 - kb_lo;
   const int max_start = doc_start_of(a.cu, a.num_seqs, m_last);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i) mbar_init(bars + 8u * i, 1);
-    mbar_init(ds_full(0), 128);
-    mbar_init(ds_full(1), 128);
+    mbar_init(ds_full, 256);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -456,9 +471,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
-  const uint32_t tDQ = tmem;
+  const uint32_t tDQ = tmem, tDP = tmem + 384u;
   auto tS = [&](int b) { return tmem + 128u + 128u * b; };
-  auto tDP = [&](int b) { return tmem + 128u + 128u * b + 64u; };
 
   if (warp == kTmaWarp) {
     {
@@ -471,87 +485,88 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
         tma_load_2d_w(sbase + L::kQ + hf * (TB * 128), mq, q_full, h * D + hf * 64, m0);
         tma_load_2d_w(sbase + L::kDO + hf * (TB * 128), mdo, q_full, h * D + hf * 64, m0);
       }
-      int it = 0;
-      for (; it < T; ++it) {
-        const int s = it % NST;
-        if (!mbar_wait_warp(st_empty(s), ((it / NST) & 1) ^ 1, kErrBwd, 0x500 + s)) break;
-        const int k0 = (kb_lo + it) * SB;
-        const uint32_t stg = sbase + L::kRing + s * 2 * L::kBlk;
-        mbar_arrive_expect_tx_w(st_full(s), 2 * L::kBlk);
+      int nk = 0, nv = 0;     // blocks of K and of V issued
+      for (int j = 0; j < T; ++j) {
+        const int k0 = (kb_lo + j) * TB;
+        const int ks = j % kNK, vs = j % kNV;
+        if (!mbar_wait_warp(k_empty(ks), ((j / kNK) & 1) ^ 1, kErrBwd, 0x500 + ks)) break;
+        mbar_arrive_expect_tx_w(k_full(ks), L::kTile);
 #pragma unroll
-        for (int hf = 0; hf < D / 64; ++hf) {
-          tma_load_2d_w(stg + hf * (SB * 128), mk, st_full(s), g * D + hf * 64, k0);
-          tma_load_2d_w(stg + L::kBlk + hf * (SB * 128), mv, st_full(s), g * D + hf * 64, k0);
-        }
+        for (int hf = 0; hf < D / 64; ++hf)
+          tma_load_2d_w(sbase + L::kKRing + ks * L::kTile + hf * (TB * 128), mk, k_full(ks), g * D + hf * 64, k0);
+        ++nk;
+        if (!mbar_wait_warp(v_empty(vs), ((j / kNV) & 1) ^ 1, kErrBwd, 0x508 + vs)) break;
+        mbar_arrive_expect_tx_w(v_full(vs), L::kTile);
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf)
+          tma_load_2d_w(sbase + L::kVRing + vs * L::kTile + hf * (TB * 128), mv, v_full(vs), g * D + hf * 64, k0);
+        ++nv;
       }
-      for (int k = it > NST ? it - NST : 0; k < it; ++k)
-        mbar_wait_drain_w(st_full(k % NST), (k / NST) & 1, kErrBwd, 0x5f0);
+      // Drain: every issued load must land before the CTA can exit.
+      for (int k = nk > kNK ? nk - kNK : 0; k < nk; ++k)
+        mbar_wait_drain_w(k_full(k % kNK), (k / kNK) & 1, kErrBwd, 0x5f0);
+      for (int k = nv > kNV ? nv - kNV : 0; k < nv; ++k)
+        mbar_wait_drain_w(v_full(k % kNV), (k / kNV) & 1, kErrBwd, 0x5f2);
       mbar_wait_drain_w(q_full, 0, kErrBwd, 0x5f1);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
     {
-      // Tensor-pipe order: S(i+1) dP(i+1) | dQ(i) | dP(i+2) S(i+2) | dQ(i+1) ...
-      // dP(i+2) does not touch the columns dQ(i) reads (dS sits over S), so it
-      // is issued at once; only S(i+2) waits for dQ(i) to have read dS.
-      constexpr uint32_t idS = idesc_bf16_f32(TB, SB, 0, 0);
+      constexpr uint32_t idS = idesc_bf16_f32(TB, TB, 0, 0);
       constexpr uint32_t idA = idesc_bf16_f32(TB, D, 0, 1);
       bool ok = mbar_wait_warp(q_full, 0, kErrBwd, 0x600);
       tc_fence_after();
-      auto stage = [&](int it) { return sbase + L::kRing + (it % NST) * 2 * L::kBlk; };
-      // Descriptors built once; per MMA only a constant offset is added.
       const uint64_t dQ0 = smem_desc_sw128(sbase + L::kQ, 16, 1024);
       const uint64_t dDO0 = smem_desc_sw128(sbase + L::kDO, 16, 1024);
-      const uint64_t dRing0 = smem_desc_sw128(sbase + L::kRing, 16, 1024);
-      const uint64_t dRingMN0 = smem_desc_sw128(sbase + L::kRing, SB * 128, 1024);
-      auto issue_s = [&](int it) {
-        const uint64_t kd = desc_adv(dRing0, (it % NST) * 2 * L::kBlk);
+      const uint64_t dK0 = smem_desc_sw128(sbase + L::kKRing, 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(sbase + L::kVRing, 16, 1024);
+      const uint64_t dKmn0 = smem_desc_sw128(sbase + L::kKRing, TB * 128, 1024);
+      auto issue_s = [&](int it) -> bool {
+        if (!mbar_wait_warp(k_full(it % kNK), (it / kNK) & 1, kErrBwd, 0x610)) return false;
+        tc_fence_after();
+        const uint64_t kd = desc_adv(dK0, (it % kNK) * L::kTile);
         const uint32_t dst = tS(it & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qo = (kk / 4) * (TB * 128) + (kk % 4) * 32;
-          const uint32_t ko = (kk / 4) * (SB * 128) + (kk % 4) * 32;
-          mma_ss_w(dst, desc_adv(dQ0, qo), desc_adv(kd, ko), idS, kk > 0 ? 1u : 0u);
+          const uint32_t o = (kk / 4) * (TB * 128) + (kk % 4) * 32;
+          mma_ss_w(dst, desc_adv(dQ0, o), desc_adv(kd, o), idS, kk > 0 ? 1u : 0u);
         }
         mma_commit_w(s_full(it & 1));
+        return true;
       };
-      auto issue_dp = [&](int it) {
-        const uint64_t vd = desc_adv(dRing0, (it % NST) * 2 * L::kBlk + L::kBlk);
-        const uint32_t dst = tDP(it & 1);
+      auto issue_dp = [&](int it) -> bool {
+        if (!mbar_wait_warp(v_full(it % kNV), (it / kNV) & 1, kErrBwd, 0x611)) return false;
+        tc_fence_after();
+        const uint64_t vd = desc_adv(dV0, (it % kNV) * L::kTile);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qo = (kk / 4) * (TB * 128) + (kk % 4) * 32;
-          const uint32_t ko = (kk / 4) * (SB * 128) + (kk % 4) * 32;
-          mma_ss_w(dst, desc_adv(dDO0, qo), desc_adv(vd, ko), idS, kk > 0 ? 1u : 0u);
+          const uint32_t o = (kk / 4) * (TB * 128) + (kk % 4) * 32;
+          mma_ss_w(tDP, desc_adv(dDO0, o), desc_adv(vd, o), idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit_w(dp_full(it & 1));
+        mma_commit_w(dp_full);
+        return true;
       };
-      for (int it = 0; it < 2 && it < T && ok; ++it) {
-        if (!mbar_wait_warp(st_full(it % NST), (it / NST) & 1, kErrBwd, 0x610)) { ok = false; break; }
-        tc_fence_after();
-        issue_s(it);
-        issue_dp(it);
-      }
+      if (ok && T > 0) ok = issue_s(0) && issue_dp(0);
+      if (ok && T > 1) ok = issue_s(1);
       for (int it = 0; it < T && ok; ++it) {
         const int b = it & 1;
-        const uint32_t stg = stage(it);
-        if (!mbar_wait_warp(ds_full(b), (it >> 1) & 1, kErrBwd, 0x630)) { ok = false; break; }
+        if (!mbar_wait_warp(ds_full, it & 1, kErrBwd, 0x630)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t kb = desc_adv(dRingMN0, stg - (sbase + L::kRing));
-        const uint32_t aS = tS(b);
+        mma_commit_w(v_empty(it % kNV));                 // dP(it) has completed: V(it) is free
+        if (it + 1 < T && !issue_dp(it + 1)) { ok = false; break; }
+        // dQ += dS K: keys [0,64) from S columns [0,32), keys [64,128) from [64,96)
+        const uint64_t kmn = desc_adv(dKmn0, (it % kNK) * L::kTile);
 #pragma unroll
-        for (int kk = 0; kk < SB / 16; ++kk)
-          mma_ts_w(tDQ, aS + kk * 8, desc_adv(kb, kk * 2048), idA, (it > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < TB / 16; ++kk) {
+          const uint32_t acol = (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8;
+          mma_ts_w(tDQ, tS(b) + acol, desc_adv(kmn, kk * 2048), idA, (it > 0 || kk > 0) ? 1u : 0u);
+        }
         mma_commit_w(dq_done(b));
-        mma_commit_w(st_empty(it % NST));
-        const int nx = it + 2;
-        if (nx < T) {
-          if (!mbar_wait_warp(st_full(nx % NST), (nx / NST) & 1, kErrBwd, 0x610)) { ok = false; break; }
-          tc_fence_after();
-          issue_dp(nx);
+        mma_commit_w(k_empty(it % kNK));
+        if (it + 2 < T) {
           if (!mbar_wait_warp(dq_done(b), (it >> 1) & 1, kErrBwd, 0x620)) { ok = false; break; }
           tc_fence_after();
-          issue_s(nx);
+          if (!issue_s(it + 2)) { ok = false; break; }
         }
       }
       mma_commit_w(acc_done);
@@ -560,8 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
     __syncwarp();
   } else {
     // ------------------------------------------------------------ elementwise
-    const int b = warp >> 2;
-    const int lrow = 32 * (warp & 3) + lane;            // TMEM lane = query row
+    const int wg = warp >> 2;                            // key half of every block
+    const int lrow = 32 * (warp & 3) + lane;             // TMEM lane = query row
     const uint32_t loff = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const int i = m0 + lrow;
     const int ic = min(i, N - 1);
@@ -570,22 +585,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
     const float lse2_i = a.lse2[vo];
     const float D_i = a.Dv[vo];
     const float sl2 = a.scale_log2;
+    const uint32_t col0 = 64u * wg;
     bool ok = true;
-    for (int it = b; it < T; it += 2) {
-      const int k0 = (kb_lo + it) * SB;
-      if (!mbar_wait_warp(s_full(b), (it >> 1) & 1, kErrBwd, 0x700)) { ok = false; break; }
+    for (int it = 0; it < T; ++it) {
+      const int k0 = (kb_lo + it) * TB + 64 * wg;
+      const uint32_t sb = tS(it & 1) + col0 + loff;
+      if (!mbar_wait_warp(s_full(it & 1), (it >> 1) & 1, kErrBwd, 0x700)) { ok = false; break; }
       tc_fence_after();
-      uint32_t pv[SB], dp[SB];
-      tmem_ld32(tS(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
-      tmem_ld32(tS(b) + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
-      if (!mbar_wait_warp(dp_full(b), (it >> 1) & 1, kErrBwd, 0x710)) { ok = false; break; }
+      uint32_t pv[64], dp[64];
+      tmem_ld32(sb, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
+      tmem_ld32(sb + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
+      if (!mbar_wait_warp(dp_full, it & 1, kErrBwd, 0x710)) { ok = false; break; }
       tc_fence_after();
-      tmem_ld32(tDP(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-      tmem_ld32(tDP(b) + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      tmem_ld32(tDP + col0 + loff, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+      tmem_ld32(tDP + col0 + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
       tmem_wait_ld();
-      const bool need_mask = (k0 + SB - 1 > m0) || (k0 < max_start);
+      const bool need_mask = (k0 + 63 > m0) || (k0 < max_start);
 #pragma unroll
-      for (int c = 0; c < SB; c += 2) {
+      for (int c = 0; c < 64; c += 2) {
         float p0 = ex2_approx(u2f(pv[c]) * sl2 - lse2_i);
         float p1 = ex2_approx(u2f(pv[c + 1]) * sl2 - lse2_i);
         if (need_mask) {
@@ -595,17 +612,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
         }
         pv[c / 2] = pack_bf16x2(p0 * (u2f(dp[c]) - D_i), p1 * (u2f(dp[c + 1]) - D_i));   // in place
       }
-      tmem_st32(tS(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
+      tmem_st32(sb, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(ds_full(b));
+      mbar_arrive(ds_full);
     }
-    // epilogue: each warpgroup writes half of the dQ row (columns b*D/2 ...)
+    // epilogue: each warpgroup writes half of the dQ row (columns wg*D/2 ...)
     if (ok && mbar_wait_warp(acc_done, 0, kErrBwd, 0x720)) {
       tc_fence_after();
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dq.p[r]) + (static_cast<int64_t>(i) * a.Hl + h) * D;
 #pragma unroll 1
-      for (int c4 = b * (D / 64); c4 < (b + 1) * (D / 64); ++c4) {
+      for (int c4 = wg * (D / 64); c4 < (wg + 1) * (D / 64); ++c4) {
         uint32_t v[32];
         tmem_ld32(tDQ + loff + c4 * 32, v);
         tmem_wait_ld();
@@ -721,7 +738,7 @@ cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void
     if (!encode(enc, &ka.tq[r], q[r], s.N, qe, SB) || !encode(enc, &ka.tdo[r], dO[r], s.N, qe, SB) ||
         !encode(enc, &ka.tk[r], k[r], s.N, ke, TB) || !encode(enc, &ka.tv[r], v[r], s.N, ke, TB) ||
         !encode(enc, &qa.tq[r], q[r], s.N, qe, TB) || !encode(enc, &qa.tdo[r], dO[r], s.N, qe, TB) ||
-        !encode(enc, &qa.tk[r], k[r], s.N, ke, SB) || !encode(enc, &qa.tv[r], v[r], s.N, ke, SB))
+        !encode(enc, &qa.tk[r], k[r], s.N, ke, TB) || !encode(enc, &qa.tv[r], v[r], s.N, ke, TB))
       return cudaErrorInvalidValue;
     ka.dk.p[r] = dk[r];
     ka.dv.p[r] = dv[r];
