@@ -329,6 +329,35 @@ def main():
         roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hp, "unit": "GB/s",
                 "frac": achieved / hp, "traffic": None, "peak_source": f"{peak_src} hbm_gbs"}
 
+    # ---------------------------------------------------------------- fused layer (all-to-alls in the kernels)
+    fused = None
+    if w.backward and (N // P) % 128 == 0:
+        lf = U.UlyssesLayer(N, P, H, H_kv, d, device=dev, cu_seqlens=cu, fused=True)
+
+        def fused_step(ev=None):
+            if ev: ev[0].record(stream)
+            U.ulysses_attn_fwd_seq(q, k, v, o, lf.lse, N, P, H, H_kv, d, cu)
+            if ev: ev[1].record(stream)
+            U.ulysses_attn_bwd_seq(q, k, v, o, lf.lse, do, dq, dk, dv, N, P, H, H_kv, d, lf.workspace, cu)
+            if ev: ev[2].record(stream)
+
+        for _ in range(args.warmup):
+            fused_step()
+        torch.cuda.synchronize()
+        fev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for s_ in range(args.steps):
+            fused_step(fev[s_])
+        torch.cuda.synchronize()
+        f_fwd_ms = sum(e[0].elapsed_time(e[1]) for e in fev) / args.steps
+        f_bwd_ms = sum(e[1].elapsed_time(e[2]) for e in fev) / args.steps
+        f_ms, f_val = aggregate_over_ranks(f_fwd_ms + f_bwd_ms, N, world, reduce_max)
+        fused = {"value": f_val, "unit": "tokens/s", "ms_per_step": f_ms, "attn_fwd_seq_ms": f_fwd_ms,
+                 "attn_bwd_seq_ms": f_bwd_ms, "gpu_launches_per_step": 1 + 3,
+                 "note": "all-to-alls folded into the attention kernels' addressing (no permute launches)"}
+        del lf
+
     # ---------------------------------------------------------------- end to end through the public API
     e2e = None
     if not args.no_e2e:
@@ -388,7 +417,7 @@ def main():
                        "parallelism": f"{P} virtual ranks per GPU; {world} independent replica(s)"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk, "detail": detail,
+            "clocks": clk, "detail": detail, "fused": fused,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

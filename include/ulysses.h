@@ -114,6 +114,25 @@ ULY_API uly_status ulysses_attn_fwd(
     float softmax_scale, int causal,
     int rank_lo, int rank_hi, cudaStream_t stream);
 
+/* Fused layer forward: the seq->head all-to-all, ulysses_attn_fwd and the
+ * head->seq all-to-all in ONE launch. The kernel fetches each rank's Q/K/V
+ * tiles straight from the sequence shards (rank r's heads are a column slice
+ * of every shard row) and stores O straight into the sequence shards, so no
+ * head-sharded copy is ever written: the exchange happens in the addressing.
+ * Results are bit-identical to the three separate calls.
+ *   q_seq (H heads), k_seq, v_seq (H_kv heads): all P sequence shards,
+ *   o_seq: all P sequence shards (only the head columns of ranks
+ *   [rank_lo, rank_hi) are written), lse_head: per rank in range, [H/P, N].
+ * Needs (N/P) % 128 == 0 (a 128-token tile never straddles two shards);
+ * otherwise ULY_ERR_UNSUPPORTED. Everything else as ulysses_attn_fwd. */
+ULY_API uly_status ulysses_attn_fwd_seq(
+    const void* const* q_seq, const void* const* k_seq, const void* const* v_seq,
+    void* const* o_seq, float* const* lse_head,
+    int64_t N, int P, int H, int H_kv, int d,
+    const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
+    float softmax_scale, int causal,
+    int rank_lo, int rank_hi, cudaStream_t stream);
+
 /* Bytes of device workspace ulysses_attn_bwd needs for these sizes: per
  * (rank, query head, row padded to a multiple of 128) the fp32 values
  * lse_i*log2(e) and D_i = dO_i . O_i, for all P ranks. Returns 0 for an
@@ -136,6 +155,22 @@ ULY_API uly_status ulysses_attn_bwd(
     const void* const* q_head, const void* const* k_head, const void* const* v_head,
     const void* const* o_head, const float* const* lse_head, const void* const* do_head,
     void* const* dq_head, void* const* dk_head, void* const* dv_head,
+    int64_t N, int P, int H, int H_kv, int d,
+    const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
+    float softmax_scale,
+    void* workspace, size_t workspace_bytes,
+    int rank_lo, int rank_hi, cudaStream_t stream);
+
+/* Fused layer backward: the seq->head all-to-all of dO, ulysses_attn_bwd and
+ * the head->seq all-to-all of dQ, dK, dV, reading Q, K, V, O, dO from the
+ * sequence shards and writing dQ, dK, dV into them (all arrays: P sequence
+ * shards; lse_head: per rank in range, from ulysses_attn_fwd_seq or
+ * ulysses_attn_fwd). Workspace as ulysses_attn_bwd. Bit-identical to the
+ * separate calls. Needs (N/P) % 128 == 0; otherwise ULY_ERR_UNSUPPORTED. */
+ULY_API uly_status ulysses_attn_bwd_seq(
+    const void* const* q_seq, const void* const* k_seq, const void* const* v_seq,
+    const void* const* o_seq, const float* const* lse_head, const void* const* do_seq,
+    void* const* dq_seq, void* const* dk_seq, void* const* dv_seq,
     int64_t N, int P, int H, int H_kv, int d,
     const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
     float softmax_scale,

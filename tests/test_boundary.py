@@ -102,3 +102,15 @@ def test_bwd_validation_and_workspace_size(L):
     need = L.ulysses_attn_bwd_workspace_size(256, P, 8, 8, 64)
     assert L.ulysses_attn_bwd(p, p, p, p, p, p, p, p, p, 256, P, 8, 8, 64, None, 0, 0, 0.0,
                               ctypes.c_void_p(GOOD + 16), need, 0, P, None) == 1
+
+
+def test_fused_entry_points_need_shards_of_128_tokens(L):
+    P = 2
+    p = _arr([GOOD] * P)
+    # N/P = 100: a 128-token tile would straddle two shards
+    assert L.ulysses_attn_fwd_seq(p, p, p, p, p, 200, P, 8, 8, 64, None, 0, 0, 0.0, 1, 0, P, None) == 2
+    assert L.ulysses_attn_bwd_seq(p, p, p, p, p, p, p, p, p, 200, P, 8, 8, 64, None, 0, 0, 0.0,
+                                  ctypes.c_void_p(GOOD), 1 << 20, 0, P, None) == 2
+    # every sequence shard must be given, even for a partial rank range
+    half = _arr([GOOD, 0])
+    assert L.ulysses_attn_fwd_seq(half, p, p, p, p, 256, P, 8, 8, 64, None, 0, 0, 0.0, 1, 0, 1, None) == 1

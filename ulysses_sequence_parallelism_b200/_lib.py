@@ -41,6 +41,10 @@ _SIGS = {
     "ulysses_get_device_status": [_v, ctypes.POINTER(ctypes.c_uint32)],
     "ulysses_set_wait_limit": [ctypes.c_uint32],
     "ulysses_selftest_bounded_wait": [_v],
+    "ulysses_attn_fwd_seq": [_vpp, _vpp, _vpp, _vpp, _fpp, _i64, _i, _i, _i, _i, _v, _i, _i, ctypes.c_float, _i,
+                             _i, _i, _v],
+    "ulysses_attn_bwd_seq": [_vpp, _vpp, _vpp, _vpp, _fpp, _vpp, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _v, _i,
+                             _i, ctypes.c_float, _v, ctypes.c_size_t, _i, _i, _v],
     "ulysses_attn_bwd_noalloc": [_vpp, _vpp, _vpp, _vpp, _fpp, _vpp, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _v, _i,
                                  _i, ctypes.c_float, _i, _i, _v],
 }

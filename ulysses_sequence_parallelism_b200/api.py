@@ -20,7 +20,7 @@ from ._lib import lib, check, UlyssesError, MAX_RANKS
 __all__ = [
     "ulysses_a2a_seq_to_head", "ulysses_a2a_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_bwd",
     "ulysses_attn_bwd_workspace_size", "ulysses_get_device_status", "ulysses_set_wait_limit",
-    "ulysses_selftest_bounded_wait", "UlyssesLayer",
+    "ulysses_selftest_bounded_wait", "ulysses_attn_fwd_seq", "ulysses_attn_bwd_seq", "UlyssesLayer",
 ]
 
 
@@ -82,6 +82,30 @@ def ulysses_attn_fwd(q_head, k_head, v_head, o_head, lse_head, N, P, H, H_kv, d,
     check("ulysses_attn_fwd", code)
 
 
+def ulysses_attn_fwd_seq(q_seq, k_seq, v_seq, o_seq, lse_head, N, P, H, H_kv, d, cu_seqlens=None,
+                         max_seqlen=0, softmax_scale=0.0, causal=1, rank_lo=0, rank_hi=None, stream=None):
+    cu, ns = _cu(cu_seqlens)
+    code = lib().ulysses_attn_fwd_seq(
+        _ptrs(q_seq, P), _ptrs(k_seq, P), _ptrs(v_seq, P), _ptrs(o_seq, P), _ptrs(lse_head, P, torch.float32),
+        N, P, H, H_kv, d, cu, ns, max_seqlen, float(softmax_scale), causal, rank_lo,
+        P if rank_hi is None else rank_hi, _stream(stream))
+    check("ulysses_attn_fwd_seq", code)
+
+
+def ulysses_attn_bwd_seq(q_seq, k_seq, v_seq, o_seq, lse_head, do_seq, dq_seq, dk_seq, dv_seq, N, P, H, H_kv, d,
+                         workspace: torch.Tensor, cu_seqlens=None, max_seqlen=0, softmax_scale=0.0, rank_lo=0,
+                         rank_hi=None, stream=None):
+    cu, ns = _cu(cu_seqlens)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    code = lib().ulysses_attn_bwd_seq(
+        _ptrs(q_seq, P), _ptrs(k_seq, P), _ptrs(v_seq, P), _ptrs(o_seq, P), _ptrs(lse_head, P, torch.float32),
+        _ptrs(do_seq, P), _ptrs(dq_seq, P), _ptrs(dk_seq, P), _ptrs(dv_seq, P), N, P, H, H_kv, d, cu, ns,
+        max_seqlen, float(softmax_scale), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), rank_lo, P if rank_hi is None else rank_hi, _stream(stream))
+    check("ulysses_attn_bwd_seq", code)
+
+
 def ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d) -> int:
     return int(lib().ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d))
 
@@ -126,7 +150,7 @@ class UlyssesLayer:
 
     def __init__(self, N: int, P: int, H: int, H_kv: int, d: int, device="cuda", cu_seqlens=None,
                  max_seqlen: int = 0, softmax_scale: float = 0.0, backward: bool = True,
-                 rank_sequential: bool = False):
+                 rank_sequential: bool = False, fused: bool = False):
         if P > MAX_RANKS:
             raise ValueError(f"P <= {MAX_RANKS}")
         self.N, self.P, self.H, self.H_kv, self.d = N, P, H, H_kv, d
@@ -134,11 +158,18 @@ class UlyssesLayer:
         self.max_seqlen = max_seqlen
         self.scale = softmax_scale
         self.rank_sequential = rank_sequential
+        # fused: the all-to-alls happen inside the attention kernels' addressing
+        # (ulysses_attn_fwd_seq / ulysses_attn_bwd_seq); no head-sharded copies.
+        self.fused = fused
+        if fused and (rank_sequential or (N // P) % 128 != 0):
+            raise ValueError("the fused layer needs all ranks at once and N/P a multiple of 128")
         bf, f32 = torch.bfloat16, torch.float32
         nb = 1 if rank_sequential else P      # rank-sequential: one rank's head buffers, reused
+        if fused:
+            nb = 0
         mk = lambda hx: [torch.empty(N, hx // P, d, dtype=bf, device=device) for _ in range(nb)]
         self.q_h, self.k_h, self.v_h, self.o_h = mk(H), mk(H_kv), mk(H_kv), mk(H)
-        self.lse = [torch.empty(H // P, N, dtype=f32, device=device) for _ in range(nb)]
+        self.lse = [torch.empty(H // P, N, dtype=f32, device=device) for _ in range(P if fused else nb)]
         self.backward_enabled = backward and not rank_sequential
         if self.backward_enabled:
             self.do_h, self.dq_h, self.dk_h, self.dv_h = mk(H), mk(H), mk(H_kv), mk(H_kv)
@@ -154,7 +185,11 @@ class UlyssesLayer:
         N, P, H, H_kv, d = self.N, self.P, self.H, self.H_kv, self.d
         if o_seq is None:
             o_seq = [torch.empty_like(x) for x in q_seq]
-        if not self.rank_sequential:
+        if self.fused:
+            self._seq_in = (q_seq, k_seq, v_seq, o_seq)
+            ulysses_attn_fwd_seq(q_seq, k_seq, v_seq, o_seq, self.lse, N, P, H, H_kv, d, self.cu, self.max_seqlen,
+                                 self.scale)
+        elif not self.rank_sequential:
             ulysses_a2a_seq_to_head(q_seq, k_seq, v_seq, self.q_h, self.k_h, self.v_h, N, P, H, H_kv, d, self.cu)
             ulysses_attn_fwd(self.q_h, self.k_h, self.v_h, self.o_h, self.lse, N, P, H, H_kv, d, self.cu,
                              self.max_seqlen, self.scale)
@@ -178,6 +213,11 @@ class UlyssesLayer:
             dq_seq = [torch.empty(N // P, H, d, dtype=torch.bfloat16, device=do_seq[0].device) for _ in range(P)]
             dk_seq = [torch.empty(N // P, H_kv, d, dtype=torch.bfloat16, device=do_seq[0].device) for _ in range(P)]
             dv_seq = [torch.empty(N // P, H_kv, d, dtype=torch.bfloat16, device=do_seq[0].device) for _ in range(P)]
+        if self.fused:
+            q_seq, k_seq, v_seq, o_seq = self._seq_in
+            ulysses_attn_bwd_seq(q_seq, k_seq, v_seq, o_seq, self.lse, do_seq, dq_seq, dk_seq, dv_seq, N, P, H,
+                                 H_kv, d, self.workspace, self.cu, self.max_seqlen, self.scale)
+            return dq_seq, dk_seq, dv_seq
         ulysses_a2a_seq_to_head(do_seq, None, None, self.do_h, None, None, N, P, H, H_kv, d, self.cu)
         ulysses_attn_bwd(self.q_h, self.k_h, self.v_h, self.o_h, self.lse, self.do_h, self.dq_h, self.dk_h,
                          self.dv_h, N, P, H, H_kv, d, self.workspace, self.cu, self.max_seqlen, self.scale)

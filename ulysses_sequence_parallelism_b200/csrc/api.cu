@@ -154,6 +154,49 @@ uly_status ulysses_attn_bwd(const void* const* q_head, const void* const* k_head
                                         dv_head, workspace, stream));
 }
 
+uly_status ulysses_attn_fwd_seq(const void* const* q_seq, const void* const* k_seq, const void* const* v_seq,
+                                void* const* o_seq, float* const* lse_head, int64_t N, int P, int H, int H_kv,
+                                int d, const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
+                                float softmax_scale, int causal, int rank_lo, int rank_hi, cudaStream_t stream) {
+  (void)max_seqlen;
+  uly_status st = check_shape(N, P, H, H_kv, d, rank_lo, rank_hi);
+  if (st != ULY_OK) return st;
+  if (causal != 1 || (N / P) % 128 != 0) return ULY_ERR_UNSUPPORTED;
+  if (check_cu(cu_seqlens, num_seqs, N) != ULY_OK) return ULY_ERR_INVALID_ARG;
+  if (!ranks_ok(q_seq, 0, P) || !ranks_ok(k_seq, 0, P) || !ranks_ok(v_seq, 0, P) ||
+      !ranks_ok(reinterpret_cast<const void* const*>(o_seq), 0, P) ||
+      !ranks_ok(reinterpret_cast<const void* const*>(lse_head), rank_lo, rank_hi))
+    return ULY_ERR_INVALID_ARG;
+  uly::AttnShape s{static_cast<int>(N), P, H / P, H_kv / P, d, cu_seqlens, cu_seqlens ? num_seqs : 1,
+                   resolve_scale(softmax_scale, d), rank_lo, rank_hi};
+  return from_cuda(uly::launch_attn_fwd_seq(s, q_seq, k_seq, v_seq, o_seq, lse_head, stream));
+}
+
+uly_status ulysses_attn_bwd_seq(const void* const* q_seq, const void* const* k_seq, const void* const* v_seq,
+                                const void* const* o_seq, const float* const* lse_head, const void* const* do_seq,
+                                void* const* dq_seq, void* const* dk_seq, void* const* dv_seq, int64_t N, int P,
+                                int H, int H_kv, int d, const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
+                                float softmax_scale, void* workspace, size_t workspace_bytes, int rank_lo,
+                                int rank_hi, cudaStream_t stream) {
+  (void)max_seqlen;
+  uly_status st = check_shape(N, P, H, H_kv, d, rank_lo, rank_hi);
+  if (st != ULY_OK) return st;
+  if ((N / P) % 128 != 0) return ULY_ERR_UNSUPPORTED;
+  if (check_cu(cu_seqlens, num_seqs, N) != ULY_OK) return ULY_ERR_INVALID_ARG;
+  auto cv = [](void* const* p) { return reinterpret_cast<const void* const*>(p); };
+  if (!ranks_ok(q_seq, 0, P) || !ranks_ok(k_seq, 0, P) || !ranks_ok(v_seq, 0, P) || !ranks_ok(o_seq, 0, P) ||
+      !ranks_ok(do_seq, 0, P) || !ranks_ok(cv(dq_seq), 0, P) || !ranks_ok(cv(dk_seq), 0, P) ||
+      !ranks_ok(cv(dv_seq), 0, P) ||
+      !ranks_ok(reinterpret_cast<const void* const*>(lse_head), rank_lo, rank_hi))
+    return ULY_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ULY_ERR_INVALID_ARG;
+  if (workspace_bytes < uly::attn_bwd_workspace_bytes(N, P, H / P, d)) return ULY_ERR_INVALID_ARG;
+  uly::AttnShape s{static_cast<int>(N), P, H / P, H_kv / P, d, cu_seqlens, cu_seqlens ? num_seqs : 1,
+                   resolve_scale(softmax_scale, d), rank_lo, rank_hi};
+  return from_cuda(uly::launch_attn_bwd_seq(s, q_seq, k_seq, v_seq, o_seq, lse_head, do_seq, dq_seq, dk_seq,
+                                            dv_seq, workspace, stream));
+}
+
 const char* ulysses_status_string(uly_status s) {
   switch (s) {
     case ULY_OK: return "ok";

@@ -24,6 +24,10 @@
 //              the two warpgroups on the two key halves); dQ += dS K (TS MMA).
 // S and dP are recomputed in (3): 7 block GEMMs instead of 5, in exchange for
 // no fp32 atomics, no dQ accumulator traffic and a bit-reproducible result.
+// Layouts: as in the forward, seq == 0 reads and writes rank r's head shards
+// ([N, Hx/P, d]); seq == 1 (the fused path) maps the sequence shards
+// ([N/P, Hx, d], N/P a multiple of 128) and addresses rank r's heads as the
+// column slice at r*Hx/P*d, so no permute runs before or after.
 // Warp roles in 2 and 3: warps 0-3 / 4-7 elementwise, warp 8 TMA producer,
 // warp 9 MMA issuer (TMA and MMA warps run converged; one elected lane issues).
 // Every mbarrier wait is bounded and reports into the library error word.
@@ -44,6 +48,11 @@ constexpr int TB = 128;         // stationary block (keys in dkdv, rows in dq)
 constexpr float kLog2e = 1.4426950408889634f;
 
 ULY_DEV float u2f(uint32_t x) { return __uint_as_float(x); }
+ULY_DEV float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
 
 ULY_DEV void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -58,6 +67,7 @@ struct PrepArgs {
   float* lse2;    // [P][Hl][Npad]
   float* Dv;      // [P][Hl][Npad]
   int N, Npad, Hl, rank_lo, nranks;
+  int seq, n_loc, P;
 };
 
 template <int D>
@@ -77,9 +87,14 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ P
     h = static_cast<int>(rem - static_cast<int64_t>(i) * a.Hl);
     r = a.rank_lo + rr;
     if (i < a.N) {
-      const int64_t off = (static_cast<int64_t>(i) * a.Hl + h) * D + c * 8;
-      const uint4 ov = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o.p[r]) + off);
-      const uint4 dv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dO.p[r]) + off);
+      int buf = r;
+      int64_t off = (static_cast<int64_t>(i) * a.Hl + h) * D + c * 8;
+      if (a.seq) {
+        buf = i / a.n_loc;
+        off = (static_cast<int64_t>(i - buf * a.n_loc) * (a.Hl * a.P) + r * a.Hl + h) * D + c * 8;
+      }
+      const uint4 ov = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o.p[buf]) + off);
+      const uint4 dv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dO.p[buf]) + off);
       const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
       const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
 #pragma unroll
@@ -119,6 +134,7 @@ struct DkdvArgs {
   int N, Npad, Hl, Hkvl, group;
   float scale, scale_log2;
   int rank_lo;
+  int seq, n_loc, P;
 };
 
 template <int D>
@@ -189,14 +205,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid
 
   if (warp == kTmaWarp) {
     {
-      const CUtensorMap *mq = &a.tq[r], *mdo = &a.tdo[r], *mk = &a.tk[r], *mv = &a.tv[r];
-      if (lane == 0) tma_prefetch_desc(mq);
-      if (lane == 0) tma_prefetch_desc(mdo);
+      auto shard_of = [&](int tok) { return a.seq ? tok / a.n_loc : r; };
+      auto row_in = [&](int tok) { return a.seq ? tok - (tok / a.n_loc) * a.n_loc : tok; };
+      const int qx0 = a.seq ? r * a.Hl * D : 0, kx0 = a.seq ? (r * a.Hkvl + g) * D : g * D;
+      if (!a.seq && lane == 0) {
+        tma_prefetch_desc(&a.tq[r]);
+        tma_prefetch_desc(&a.tdo[r]);
+      }
+      const CUtensorMap *mk = &a.tk[shard_of(n0)], *mv = &a.tv[shard_of(n0)];
       mbar_arrive_expect_tx_w(kv_full, 2 * L::kKV);
 #pragma unroll
       for (int hf = 0; hf < D / 64; ++hf) {
-        tma_load_2d_w(sbase + L::kK + hf * (TB * 128), mk, kv_full, g * D + hf * 64, n0);
-        tma_load_2d_w(sbase + L::kV + hf * (TB * 128), mv, kv_full, g * D + hf * 64, n0);
+        tma_load_2d_w(sbase + L::kK + hf * (TB * 128), mk, kv_full, kx0 + hf * 64, row_in(n0));
+        tma_load_2d_w(sbase + L::kV + hf * (TB * 128), mv, kv_full, kx0 + hf * 64, row_in(n0));
       }
       int it = 0;
       for (; it < T; ++it) {
@@ -208,8 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid
         mbar_arrive_expect_tx_w(st_full(s), 2 * L::kBlk + 512);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf) {
-          tma_load_2d_w(stg + hf * (SB * 128), mq, st_full(s), h * D + hf * 64, m0);
-          tma_load_2d_w(stg + L::kBlk + hf * (SB * 128), mdo, st_full(s), h * D + hf * 64, m0);
+          tma_load_2d_w(stg + hf * (SB * 128), &a.tq[shard_of(m0)], st_full(s), qx0 + h * D + hf * 64, row_in(m0));
+          tma_load_2d_w(stg + L::kBlk + hf * (SB * 128), &a.tdo[shard_of(m0)], st_full(s), qx0 + h * D + hf * 64,
+                        row_in(m0));
         }
         const int64_t vo = (static_cast<int64_t>(r) * a.Hl + h) * a.Npad + m0;
         bulk_load_w(sbase + L::kVec + s * 512, a.lse2 + vo, SB * 4, st_full(s));
@@ -310,8 +332,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid
     for (int it = b; it < T; it += 2) {
       const int s = it % NST;
       const int m0 = (rb_lo + it % nrb) * SB;
-      const float* vl = reinterpret_cast<const float*>(sgen + L::kVec + s * 512);
-      const float* vd = vl + 64;
+      // lse*log2(e) and D of this block's 64 rows: same for every lane, read as
+      // 16-byte shared-memory broadcasts
+      const uint32_t vl = sbase + L::kVec + s * 512, vd = vl + 256;
       if (!mbar_wait_warp(st_full(s), (it / NST) & 1, kErrBwd, 0x300)) { ok = false; break; }
       if (!mbar_wait_warp(s_full(b), (it >> 1) & 1, kErrBwd, 0x310)) { ok = false; break; }
       tc_fence_after();
@@ -320,14 +343,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid
       tmem_ld32(tS(b) + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
       tmem_wait_ld();
       const bool need_mask = (m0 < n0 + TB - 1) || (m0 + SB > doc_end_first);
-      uint32_t pk[SB / 2];
+      // allowed rows of this key within the block: c in [lo, hi)  <=>  (unsigned)(c - lo) < span
+      const int lo = key - m0;
+      const uint32_t span = static_cast<uint32_t>(max(kde - key, 0));
 #pragma unroll
-      for (int c = 0; c < SB; ++c) {
-        const int row = m0 + c;
-        float p = ex2_approx(u2f(pv[c]) * sl2 - vl[c]);
-        if (need_mask && (row < key || row >= kde)) p = 0.f;
-        pv[c] = __float_as_uint(p);
+      for (int c = 0; c < SB; c += 4) {
+        const float4 l4 = ld_shared_f4(vl + 4 * c);
+        float p0 = ex2_approx(u2f(pv[c]) * sl2 - l4.x);
+        float p1 = ex2_approx(u2f(pv[c + 1]) * sl2 - l4.y);
+        float p2 = ex2_approx(u2f(pv[c + 2]) * sl2 - l4.z);
+        float p3 = ex2_approx(u2f(pv[c + 3]) * sl2 - l4.w);
+        if (need_mask) {
+          p0 = static_cast<uint32_t>(c - lo) < span ? p0 : 0.f;
+          p1 = static_cast<uint32_t>(c + 1 - lo) < span ? p1 : 0.f;
+          p2 = static_cast<uint32_t>(c + 2 - lo) < span ? p2 : 0.f;
+          p3 = static_cast<uint32_t>(c + 3 - lo) < span ? p3 : 0.f;
+        }
+        pv[c] = __float_as_uint(p0);
+        pv[c + 1] = __float_as_uint(p1);
+        pv[c + 2] = __float_as_uint(p2);
+        pv[c + 3] = __float_as_uint(p3);
       }
+      uint32_t pk[SB / 2];
 #pragma unroll
       for (int c = 0; c < SB / 2; ++c) pk[c] = pack_bf16x2(u2f(pv[2 * c]), u2f(pv[2 * c + 1]));
       tmem_st32(tS(b) + loff, pk);
@@ -341,10 +378,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid
       tmem_ld32(tDP(b) + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < SB; c += 2) {
-        const float d0 = u2f(pv[c]) * (u2f(dp[c]) - vd[c]);
-        const float d1 = u2f(pv[c + 1]) * (u2f(dp[c + 1]) - vd[c + 1]);
-        dp[c / 2] = pack_bf16x2(d0, d1);     // in place: dp[c/2] is already consumed
+      for (int c = 0; c < SB; c += 4) {
+        const float4 d4 = ld_shared_f4(vd + 4 * c);
+        const float d0 = u2f(pv[c]) * (u2f(dp[c]) - d4.x);
+        const float d1 = u2f(pv[c + 1]) * (u2f(dp[c + 1]) - d4.y);
+        const float d2 = u2f(pv[c + 2]) * (u2f(dp[c + 2]) - d4.z);
+        const float d3 = u2f(pv[c + 3]) * (u2f(dp[c + 3]) - d4.w);
+        dp[c / 2] = pack_bf16x2(d0, d1);     // in place: dp[c/2], dp[c/2+1] are already consumed
+        dp[c / 2 + 1] = pack_bf16x2(d2, d3);
       }
       tmem_st32(tDP(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
       tmem_wait_st();
@@ -356,8 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid
       tc_fence_after();
       const uint32_t src = (b == 0 ? tDV : tDK) + loff;
       const float mul = b == 0 ? 1.f : a.scale;
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(b == 0 ? a.dv.p[r] : a.dk.p[r]) +
-                           (static_cast<int64_t>(key) * a.Hkvl + g) * D;
+      const int kb = a.seq ? min(key, N - 1) / a.n_loc : r;     // clamped: rows >= N are not stored
+      const int64_t krow = a.seq ? (static_cast<int64_t>(key - kb * a.n_loc) * (a.Hkvl * a.P) + r * a.Hkvl + g)
+                                 : (static_cast<int64_t>(key) * a.Hkvl + g);
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(b == 0 ? a.dv.p[kb] : a.dk.p[kb]) + krow * D;
 #pragma unroll 1
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t v[32];
@@ -411,6 +454,7 @@ struct DqArgs {
   float scale, scale_log2;
   int rank_lo;
   int num_m_tiles;
+  int seq, n_loc, P;
 };
 
 constexpr int kNK = 3, kNV = 2;   // K and V ring depths in the dQ kernel
@@ -476,14 +520,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
 
   if (warp == kTmaWarp) {
     {
-      const CUtensorMap *mq = &a.tq[r], *mdo = &a.tdo[r], *mk = &a.tk[r], *mv = &a.tv[r];
-      if (lane == 0) tma_prefetch_desc(mk);
-      if (lane == 0) tma_prefetch_desc(mv);
+      auto shard_of = [&](int tok) { return a.seq ? tok / a.n_loc : r; };
+      auto row_in = [&](int tok) { return a.seq ? tok - (tok / a.n_loc) * a.n_loc : tok; };
+      const int qx0 = a.seq ? (r * a.Hl + h) * D : h * D, kx0 = a.seq ? (r * a.Hkvl + g) * D : g * D;
+      if (!a.seq && lane == 0) {
+        tma_prefetch_desc(&a.tk[r]);
+        tma_prefetch_desc(&a.tv[r]);
+      }
       mbar_arrive_expect_tx_w(q_full, 2 * L::kTile);
 #pragma unroll
       for (int hf = 0; hf < D / 64; ++hf) {
-        tma_load_2d_w(sbase + L::kQ + hf * (TB * 128), mq, q_full, h * D + hf * 64, m0);
-        tma_load_2d_w(sbase + L::kDO + hf * (TB * 128), mdo, q_full, h * D + hf * 64, m0);
+        tma_load_2d_w(sbase + L::kQ + hf * (TB * 128), &a.tq[shard_of(m0)], q_full, qx0 + hf * 64, row_in(m0));
+        tma_load_2d_w(sbase + L::kDO + hf * (TB * 128), &a.tdo[shard_of(m0)], q_full, qx0 + hf * 64, row_in(m0));
       }
       int nk = 0, nv = 0;     // blocks of K and of V issued
       for (int j = 0; j < T; ++j) {
@@ -493,13 +541,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
         mbar_arrive_expect_tx_w(k_full(ks), L::kTile);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf)
-          tma_load_2d_w(sbase + L::kKRing + ks * L::kTile + hf * (TB * 128), mk, k_full(ks), g * D + hf * 64, k0);
+          tma_load_2d_w(sbase + L::kKRing + ks * L::kTile + hf * (TB * 128), &a.tk[shard_of(k0)], k_full(ks),
+                        kx0 + hf * 64, row_in(k0));
         ++nk;
         if (!mbar_wait_warp(v_empty(vs), ((j / kNV) & 1) ^ 1, kErrBwd, 0x508 + vs)) break;
         mbar_arrive_expect_tx_w(v_full(vs), L::kTile);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf)
-          tma_load_2d_w(sbase + L::kVRing + vs * L::kTile + hf * (TB * 128), mv, v_full(vs), g * D + hf * 64, k0);
+          tma_load_2d_w(sbase + L::kVRing + vs * L::kTile + hf * (TB * 128), &a.tv[shard_of(k0)], v_full(vs),
+                        kx0 + hf * 64, row_in(k0));
         ++nv;
       }
       // Drain: every issued load must land before the CTA can exit.
@@ -620,7 +670,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
     // epilogue: each warpgroup writes half of the dQ row (columns wg*D/2 ...)
     if (ok && mbar_wait_warp(acc_done, 0, kErrBwd, 0x720)) {
       tc_fence_after();
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dq.p[r]) + (static_cast<int64_t>(i) * a.Hl + h) * D;
+      const int qb = a.seq ? ic / a.n_loc : r;           // ic clamped: rows >= N are not stored
+      const int64_t qrow = a.seq ? (static_cast<int64_t>(ic - qb * a.n_loc) * (a.Hl * a.P) + r * a.Hl + h)
+                                 : (static_cast<int64_t>(i) * a.Hl + h);
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dq.p[qb]) + qrow * D;
 #pragma unroll 1
       for (int c4 = wg * (D / 64); c4 < (wg + 1) * (D / 64); ++c4) {
         uint32_t v[32];
@@ -714,16 +767,46 @@ size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d) {
   return 2 * static_cast<size_t>(P) * Hl * npad * sizeof(float);
 }
 
+namespace bwd_sm100 {
+// Fills everything but the per-buffer pointers and tensor maps, then launches.
+cudaError_t launch_common(const AttnShape& s, PrepArgs& pa, DkdvArgs& ka, DqArgs& qa, void* workspace, int seq,
+                          cudaStream_t stream) {
+  const int Npad = padded_rows(s.N);
+  float* lse2 = static_cast<float*>(workspace);
+  float* Dv = lse2 + static_cast<size_t>(s.P) * s.Hl * Npad;
+  pa.lse2 = lse2;
+  pa.Dv = Dv;
+  pa.N = s.N;
+  pa.Npad = Npad;
+  pa.Hl = s.Hl;
+  pa.rank_lo = s.rank_lo;
+  pa.nranks = s.rank_hi - s.rank_lo;
+  pa.seq = ka.seq = qa.seq = seq;
+  pa.n_loc = ka.n_loc = qa.n_loc = s.N / s.P;
+  pa.P = ka.P = qa.P = s.P;
+  ka.lse2 = qa.lse2 = lse2;
+  ka.Dv = qa.Dv = Dv;
+  ka.cu = qa.cu = s.cu_seqlens;
+  ka.num_seqs = qa.num_seqs = s.num_seqs;
+  ka.N = qa.N = s.N;
+  ka.Npad = qa.Npad = Npad;
+  ka.Hl = qa.Hl = s.Hl;
+  ka.Hkvl = qa.Hkvl = s.Hkvl;
+  ka.group = qa.group = s.Hl / s.Hkvl;
+  ka.scale = qa.scale = s.scale;
+  ka.scale_log2 = qa.scale_log2 = s.scale * kLog2e;
+  ka.rank_lo = qa.rank_lo = s.rank_lo;
+  qa.num_m_tiles = (s.N + TB - 1) / TB;
+  return s.d == 64 ? launch_all<64>(s, pa, ka, qa, stream) : launch_all<128>(s, pa, ka, qa, stream);
+}
+}  // namespace bwd_sm100
+
 cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void* const* k, const void* const* v,
                             const void* const* o, const float* const* lse, const void* const* dO, void* const* dq,
                             void* const* dk, void* const* dv, void* workspace, cudaStream_t stream) {
   using namespace bwd_sm100;
   EncodeTiledFn enc = get_encode();
   if (enc == nullptr) return cudaErrorNotSupported;
-  const int Npad = padded_rows(s.N);
-  float* lse2 = static_cast<float*>(workspace);
-  float* Dv = lse2 + static_cast<size_t>(s.P) * s.Hl * Npad;
-
   PrepArgs pa;
   memset(&pa, 0, sizeof(pa));
   DkdvArgs ka;
@@ -744,28 +827,38 @@ cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void
     ka.dv.p[r] = dv[r];
     qa.dq.p[r] = dq[r];
   }
-  pa.lse2 = lse2;
-  pa.Dv = Dv;
-  pa.N = s.N;
-  pa.Npad = Npad;
-  pa.Hl = s.Hl;
-  pa.rank_lo = s.rank_lo;
-  pa.nranks = s.rank_hi - s.rank_lo;
+  return launch_common(s, pa, ka, qa, workspace, 0, stream);
+}
 
-  ka.lse2 = qa.lse2 = lse2;
-  ka.Dv = qa.Dv = Dv;
-  ka.cu = qa.cu = s.cu_seqlens;
-  ka.num_seqs = qa.num_seqs = s.num_seqs;
-  ka.N = qa.N = s.N;
-  ka.Npad = qa.Npad = Npad;
-  ka.Hl = qa.Hl = s.Hl;
-  ka.Hkvl = qa.Hkvl = s.Hkvl;
-  ka.group = qa.group = s.Hl / s.Hkvl;
-  ka.scale = qa.scale = s.scale;
-  ka.scale_log2 = qa.scale_log2 = s.scale * kLog2e;
-  ka.rank_lo = qa.rank_lo = s.rank_lo;
-  qa.num_m_tiles = (s.N + TB - 1) / TB;
-  return s.d == 64 ? launch_all<64>(s, pa, ka, qa, stream) : launch_all<128>(s, pa, ka, qa, stream);
+cudaError_t launch_attn_bwd_seq(const AttnShape& s, const void* const* q_seq, const void* const* k_seq,
+                                const void* const* v_seq, const void* const* o_seq, const float* const* lse,
+                                const void* const* do_seq, void* const* dq_seq, void* const* dk_seq,
+                                void* const* dv_seq, void* workspace, cudaStream_t stream) {
+  using namespace bwd_sm100;
+  EncodeTiledFn enc = get_encode();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  PrepArgs pa;
+  memset(&pa, 0, sizeof(pa));
+  DkdvArgs ka;
+  memset(&ka, 0, sizeof(ka));
+  DqArgs qa;
+  memset(&qa, 0, sizeof(qa));
+  const int64_t n = s.N / s.P;
+  const int64_t qe = static_cast<int64_t>(s.Hl) * s.P * s.d, ke = static_cast<int64_t>(s.Hkvl) * s.P * s.d;
+  for (int p = 0; p < s.P; ++p) {
+    pa.o.p[p] = o_seq[p];
+    pa.dO.p[p] = do_seq[p];
+    if (!encode(enc, &ka.tq[p], q_seq[p], n, qe, SB) || !encode(enc, &ka.tdo[p], do_seq[p], n, qe, SB) ||
+        !encode(enc, &ka.tk[p], k_seq[p], n, ke, TB) || !encode(enc, &ka.tv[p], v_seq[p], n, ke, TB) ||
+        !encode(enc, &qa.tq[p], q_seq[p], n, qe, TB) || !encode(enc, &qa.tdo[p], do_seq[p], n, qe, TB) ||
+        !encode(enc, &qa.tk[p], k_seq[p], n, ke, TB) || !encode(enc, &qa.tv[p], v_seq[p], n, ke, TB))
+      return cudaErrorInvalidValue;
+    ka.dk.p[p] = dk_seq[p];
+    ka.dv.p[p] = dv_seq[p];
+    qa.dq.p[p] = dq_seq[p];
+  }
+  for (int r = s.rank_lo; r < s.rank_hi; ++r) pa.lse.p[r] = lse[r];
+  return launch_common(s, pa, ka, qa, workspace, 1, stream);
 }
 
 }  // namespace uly

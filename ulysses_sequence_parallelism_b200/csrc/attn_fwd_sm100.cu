@@ -40,6 +40,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O when the max grows by > 2^8
 
+// Two source/destination layouts share the kernel:
+//  head layout (seq == 0): tq/tk/tv[r] map rank r's head shard [N, Hl*d]; o.p[r]
+//    is rank r's head-sharded O.
+//  sequence layout (seq == 1, the fused path): tq/tk/tv[p] map sequence shard p
+//    [n, H*d] (n = N/P, a multiple of 128, so no 128-token tile straddles two
+//    shards) and rank r's heads are the column slice starting at r*Hl*d;
+//    o.p[p] is sequence shard p of O. The all-to-alls disappear into the
+//    addressing: each tile is fetched from, and stored to, where it lives.
 struct FwdArgs {
   CUtensorMap tq[kMaxRanks];
   CUtensorMap tk[kMaxRanks];
@@ -52,6 +60,9 @@ struct FwdArgs {
   float scale_log2;
   int rank_lo;
   int num_m_blocks;   // blocks of 2*BM rows
+  int seq;            // 1: sequence layout (see above)
+  int n_loc;          // N / P
+  int P;
 };
 
 template <int D>
@@ -136,33 +147,40 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     {
-      const CUtensorMap* mq = &a.tq[r];
-      const CUtensorMap* mk = &a.tk[r];
-      const CUtensorMap* mv = &a.tv[r];
-      if (lane == 0) tma_prefetch_desc(mq);
-      if (lane == 0) tma_prefetch_desc(mk);
-      if (lane == 0) tma_prefetch_desc(mv);
+      // Map and coordinates of a token range: its shard and row within it.
+      const int qx0 = a.seq ? (r * a.Hl + h) * D : h * D;
+      const int kx0 = a.seq ? (r * a.Hkvl + g) * D : g * D;
+      auto shard_of = [&](int tok) { return a.seq ? tok / a.n_loc : r; };
+      auto row_in = [&](int tok) { return a.seq ? tok - (tok / a.n_loc) * a.n_loc : tok; };
+      if (!a.seq && lane == 0) {
+        tma_prefetch_desc(&a.tq[r]);
+        tma_prefetch_desc(&a.tk[r]);
+        tma_prefetch_desc(&a.tv[r]);
+      }
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (!active[t]) continue;
         mbar_arrive_expect_tx_w(q_full(t), L::kQTile);
+        const CUtensorMap* mq = &a.tq[shard_of(first_row[t])];
+        const int qy = row_in(first_row[t]);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf)
-          tma_load_2d_w(sQ + t * L::kQTile + hf * (BM * 128), mq, q_full(t), h * D + hf * 64, first_row[t]);
+          tma_load_2d_w(sQ + t * L::kQTile + hf * (BM * 128), mq, q_full(t), qx0 + hf * 64, qy);
       }
       uint32_t it = 0;
       bool ok = true;
       for (int jb = jb_lo; jb < jb_hi && ok; ++jb) {
+        const int kp = shard_of(jb * BN), ky = row_in(jb * BN);
 #pragma unroll
         for (int kind = 0; kind < 2; ++kind, ++it) {
           const int s = it % NSTAGE;
           const uint32_t ph = (it / NSTAGE) & 1u;
           if (!mbar_wait_warp(kv_empty(s), ph ^ 1u, kErrFwd, 0x100 + s)) { ok = false; break; }
           mbar_arrive_expect_tx_w(kv_full(s), L::kKV);
-          const CUtensorMap* m = kind == 0 ? mk : mv;
+          const CUtensorMap* m = kind == 0 ? &a.tk[kp] : &a.tv[kp];
 #pragma unroll
           for (int hf = 0; hf < D / 64; ++hf)
-            tma_load_2d_w(sRing + s * L::kKV + hf * (BN * 128), m, kv_full(s), g * D + hf * 64, jb * BN);
+            tma_load_2d_w(sRing + s * L::kKV + hf * (BN * 128), m, kv_full(s), kx0 + hf * 64, ky);
         }
       }
       // Drain: every issued load must land before the CTA can exit.
@@ -369,7 +387,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
       if (ok && cnt > 0 && mbar_wait_warp(pv_done(t), (cnt - 1) & 1, kErrFwd, 0x420 + t)) {
         tc_fence_after();
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o.p[r]) + (static_cast<int64_t>(i) * a.Hl + h) * D;
+        __nv_bfloat16* orow = nullptr;
+        if (row_ok) {
+          if (a.seq) {
+            const int p = i / a.n_loc;
+            orow = static_cast<__nv_bfloat16*>(a.o.p[p]) +
+                   (static_cast<int64_t>(i - p * a.n_loc) * (a.Hl * a.P) + r * a.Hl + h) * D;
+          } else {
+            orow = static_cast<__nv_bfloat16*>(a.o.p[r]) + (static_cast<int64_t>(i) * a.Hl + h) * D;
+          }
+        }
 #pragma unroll 1
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t ov[32];
@@ -439,6 +466,24 @@ cudaError_t launch_d(const FwdArgs& a, int nranks, cudaStream_t stream) {
 
 }  // namespace fwd_sm100
 
+namespace fwd_sm100 {
+cudaError_t launch_common(const AttnShape& s, FwdArgs& a, cudaStream_t stream) {
+  a.cu = s.cu_seqlens;
+  a.num_seqs = s.num_seqs;
+  a.N = s.N;
+  a.Hl = s.Hl;
+  a.Hkvl = s.Hkvl;
+  a.group = s.Hl / s.Hkvl;
+  a.scale_log2 = s.scale * kLog2e;
+  a.rank_lo = s.rank_lo;
+  a.num_m_blocks = (s.N + 2 * BM - 1) / (2 * BM);
+  a.n_loc = s.N / s.P;
+  a.P = s.P;
+  const int nranks = s.rank_hi - s.rank_lo;
+  return s.d == 64 ? launch_d<64>(a, nranks, stream) : launch_d<128>(a, nranks, stream);
+}
+}  // namespace fwd_sm100
+
 cudaError_t launch_attn_fwd(const AttnShape& s, const void* const* q, const void* const* k, const void* const* v,
                             void* const* o, float* const* lse, cudaStream_t stream) {
   using namespace fwd_sm100;
@@ -454,17 +499,29 @@ cudaError_t launch_attn_fwd(const AttnShape& s, const void* const* q, const void
     a.o.p[r] = o[r];
     a.lse.p[r] = lse[r];
   }
-  a.cu = s.cu_seqlens;
-  a.num_seqs = s.num_seqs;
-  a.N = s.N;
-  a.Hl = s.Hl;
-  a.Hkvl = s.Hkvl;
-  a.group = s.Hl / s.Hkvl;
-  a.scale_log2 = s.scale * kLog2e;
-  a.rank_lo = s.rank_lo;
-  a.num_m_blocks = (s.N + 2 * BM - 1) / (2 * BM);
-  const int nranks = s.rank_hi - s.rank_lo;
-  return s.d == 64 ? launch_d<64>(a, nranks, stream) : launch_d<128>(a, nranks, stream);
+  a.seq = 0;
+  return launch_common(s, a, stream);
+}
+
+cudaError_t launch_attn_fwd_seq(const AttnShape& s, const void* const* q_seq, const void* const* k_seq,
+                                const void* const* v_seq, void* const* o_seq, float* const* lse,
+                                cudaStream_t stream) {
+  using namespace fwd_sm100;
+  EncodeTiledFn enc = get_encode();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  FwdArgs a;
+  memset(&a, 0, sizeof(a));
+  const int64_t n = s.N / s.P;
+  const int64_t H = static_cast<int64_t>(s.Hl) * s.P, Hkv = static_cast<int64_t>(s.Hkvl) * s.P;
+  for (int p = 0; p < s.P; ++p) {
+    if (!encode_rows(enc, &a.tq[p], q_seq[p], n, H * s.d) || !encode_rows(enc, &a.tk[p], k_seq[p], n, Hkv * s.d) ||
+        !encode_rows(enc, &a.tv[p], v_seq[p], n, Hkv * s.d))
+      return cudaErrorInvalidValue;
+    a.o.p[p] = o_seq[p];
+  }
+  for (int r = s.rank_lo; r < s.rank_hi; ++r) a.lse.p[r] = lse[r];
+  a.seq = 1;
+  return launch_common(s, a, stream);
 }
 
 }  // namespace uly

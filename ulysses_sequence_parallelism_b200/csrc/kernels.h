@@ -24,6 +24,15 @@ cudaError_t launch_permute(bool seq_to_head, const void* const* src[3], void* co
 cudaError_t launch_attn_fwd(const AttnShape& s, const void* const* q, const void* const* k,
                             const void* const* v, void* const* o, float* const* lse, cudaStream_t stream);
 
+// The same kernels reading Q/K/V (and dO, O) straight from the sequence shards
+// and writing O (and dQ, dK, dV) straight into them: the permutes disappear.
+cudaError_t launch_attn_fwd_seq(const AttnShape& s, const void* const* q_seq, const void* const* k_seq,
+                                const void* const* v_seq, void* const* o_seq, float* const* lse, cudaStream_t stream);
+cudaError_t launch_attn_bwd_seq(const AttnShape& s, const void* const* q_seq, const void* const* k_seq,
+                                const void* const* v_seq, const void* const* o_seq, const float* const* lse,
+                                const void* const* do_seq, void* const* dq_seq, void* const* dk_seq,
+                                void* const* dv_seq, void* workspace, cudaStream_t stream);
+
 size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d);
 cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void* const* k,
                             const void* const* v, const void* const* o, const float* const* lse,
