@@ -438,8 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_kernel(const __grid
 //   bf16 over the start of its own S columns, and dQ += dS K is issued as two
 //   K=64 halves that read those two column ranges.
 // Tensor-pipe order per block i: dP(i+1) | dQ(i) | S(i+2): dP(i+1) goes out as
-// soon as the elementwise warps have read dP(i), so they can start block i+1
-// while dQ(i) runs.
+// soon as the elementwise warps hold dP(i) in registers (a barrier of its own,
+// before they start computing), so it runs under their arithmetic and they can
+// start block i+1 as soon as they finish block i.
 struct DqArgs {
   CUtensorMap tq[kMaxRanks];    // box 64 cols x TB rows
   CUtensorMap tdo[kMaxRanks];   // box 64 cols x TB rows
@@ -466,8 +467,9 @@ struct DqLayout {
   static constexpr uint32_t kKRing = 2 * kTile;
   static constexpr uint32_t kVRing = kKRing + kNK * kTile;
   static constexpr uint32_t kBars = kVRing + kNV * kTile;
-  // q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full[2], dp_full, ds_full, dq_done[2], acc_done
-  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 1 + 1 + 2 + 1;
+  // q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full[2], dp_full, ds_full, dq_done[2], acc_done,
+  // dp_free
+  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 1 + 1 + 2 + 1 + 1;
   static constexpr uint32_t kSlot = kBars + kNumBars * 8;
   static constexpr uint32_t kAlloc = kSlot + 16 + 1024;
 };
@@ -489,6 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
   const uint32_t ds_full = bars + 8u * (4 + 2 * kNK + 2 * kNV);
   auto dq_done = [&](int b) { return bars + 8u * (5 + 2 * kNK + 2 * kNV + b); };
   const uint32_t acc_done = bars + 8u * (7 + 2 * kNK + 2 * kNV);
+  const uint32_t dp_free = bars + 8u * (8 + 2 * kNK + 2 * kNV);
   volatile uint32_t* slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -505,6 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i) mbar_init(bars + 8u * i, 1);
     mbar_init(ds_full, 256);
+    mbar_init(dp_free, 256);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -600,10 +604,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
       if (ok && T > 1) ok = issue_s(1);
       for (int it = 0; it < T && ok; ++it) {
         const int b = it & 1;
-        if (!mbar_wait_warp(ds_full, it & 1, kErrBwd, 0x630)) { ok = false; break; }
+        if (!mbar_wait_warp(dp_free, it & 1, kErrBwd, 0x631)) { ok = false; break; }
         tc_fence_after();
         mma_commit_w(v_empty(it % kNV));                 // dP(it) has completed: V(it) is free
         if (it + 1 < T && !issue_dp(it + 1)) { ok = false; break; }
+        if (!mbar_wait_warp(ds_full, it & 1, kErrBwd, 0x630)) { ok = false; break; }
+        tc_fence_after();
         // dQ += dS K: keys [0,64) from S columns [0,32), keys [64,128) from [64,96)
         const uint64_t kmn = desc_adv(dKmn0, (it % kNK) * L::kTile);
 #pragma unroll
@@ -650,6 +656,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
       tmem_ld32(tDP + col0 + loff, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
       tmem_ld32(tDP + col0 + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(dp_free);                                // dP(it) is in registers: dP(it+1) may overwrite it
       const bool need_mask = (k0 + 63 > m0) || (k0 < max_start);
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
