@@ -196,6 +196,8 @@ def main():
     ap.add_argument("--workload", default="varlen64k", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="time the two-pass backward (bit-reproducible dQ) instead of the one-pass one")
     ap.add_argument("--tokens", type=int, default=None,
                     help="draw the workload's recipe at a smaller total N (profiling captures)")
     args = ap.parse_args()
@@ -228,7 +230,7 @@ def main():
     cu = None if cu_np is None else torch.tensor(cu_np, dtype=torch.int32, device=dev)
     P, H, H_kv, d, N = w.P, w.H, w.H_kv, w.d, w.N
     layer = U.UlyssesLayer(N, P, H, H_kv, d, device=dev, cu_seqlens=cu, backward=w.backward,
-                           rank_sequential=w.rank_sequential)
+                           rank_sequential=w.rank_sequential, deterministic=args.deterministic)
 
     def shards(x):
         n = N // P
@@ -261,7 +263,7 @@ def main():
             U.ulysses_a2a_seq_to_head(do, None, None, L.do_h, None, None, N, P, H, H_kv, d, cu)
             if ev: ev[4].record(stream)
             U.ulysses_attn_bwd(L.q_h, L.k_h, L.v_h, L.o_h, L.lse, L.do_h, L.dq_h, L.dk_h, L.dv_h, N, P, H, H_kv, d,
-                               L.workspace, cu)
+                               L.workspace, cu, deterministic=args.deterministic)
             if ev: ev[5].record(stream)
             U.ulysses_a2a_head_to_seq(L.dq_h, L.dk_h, L.dv_h, dq, dk, dv, N, P, H, H_kv, d, cu)
             if ev: ev[6].record(stream)
@@ -315,6 +317,26 @@ def main():
     if w.backward:
         detail["attn_bwd_tflops"] = f_bwd / (mean["attn_bwd"] / 1e3) / 1e12
         detail["attn_bwd_flops"] = f_bwd
+        detail["attn_bwd_mode"] = "two-pass (deterministic)" if args.deterministic else "one-pass (fp32 dQ reductions)"
+        # the other backward mode on the same buffers, for comparison (not part of the step)
+        other = not args.deterministic
+        L = layer
+        ws_other = torch.empty(U.ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, other), dtype=torch.uint8,
+                               device=dev)
+        run_other = lambda: U.ulysses_attn_bwd(L.q_h, L.k_h, L.v_h, L.o_h, L.lse, L.do_h, L.dq_h, L.dk_h, L.dv_h, N,
+                                               P, H, H_kv, d, ws_other, cu, deterministic=other)
+        for _ in range(2):
+            run_other()
+        oe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        oe[0].record(stream)
+        for _ in range(3):
+            run_other()
+        oe[1].record(stream)
+        torch.cuda.synchronize()
+        other_ms = oe[0].elapsed_time(oe[1]) / 3
+        detail["attn_bwd_other_mode"] = {"mode": "two-pass (deterministic)" if other else "one-pass",
+                                         "ms": other_ms, "tflops": f_bwd / (other_ms / 1e3) / 1e12}
+        del ws_other
     # dominant kernel by measured time
     dom = max(mean, key=mean.get)
     tensor_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
@@ -332,13 +354,15 @@ def main():
     # ---------------------------------------------------------------- fused layer (all-to-alls in the kernels)
     fused = None
     if w.backward and (N // P) % 128 == 0:
-        lf = U.UlyssesLayer(N, P, H, H_kv, d, device=dev, cu_seqlens=cu, fused=True)
+        lf = U.UlyssesLayer(N, P, H, H_kv, d, device=dev, cu_seqlens=cu, fused=True,
+                            deterministic=args.deterministic)
 
         def fused_step(ev=None):
             if ev: ev[0].record(stream)
             U.ulysses_attn_fwd_seq(q, k, v, o, lf.lse, N, P, H, H_kv, d, cu)
             if ev: ev[1].record(stream)
-            U.ulysses_attn_bwd_seq(q, k, v, o, lf.lse, do, dq, dk, dv, N, P, H, H_kv, d, lf.workspace, cu)
+            U.ulysses_attn_bwd_seq(q, k, v, o, lf.lse, do, dq, dk, dv, N, P, H, H_kv, d, lf.workspace, cu,
+                                   deterministic=args.deterministic)
             if ev: ev[2].record(stream)
 
         for _ in range(args.warmup):

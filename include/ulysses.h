@@ -133,11 +133,12 @@ ULY_API uly_status ulysses_attn_fwd_seq(
     float softmax_scale, int causal,
     int rank_lo, int rank_hi, cudaStream_t stream);
 
-/* Bytes of device workspace ulysses_attn_bwd needs for these sizes: per
- * (rank, query head, row padded to a multiple of 128) the fp32 values
- * lse_i*log2(e) and D_i = dO_i . O_i, for all P ranks. Returns 0 for an
- * invalid shape. */
-ULY_API size_t ulysses_attn_bwd_workspace_size(int64_t N, int P, int H, int H_kv, int d);
+/* Bytes of device workspace ulysses_attn_bwd needs for these sizes and this
+ * `deterministic` setting: per (rank, query head, row padded to a multiple of
+ * 128) the fp32 values lse_i*log2(e) and D_i = dO_i . O_i, for all P ranks;
+ * with deterministic == 0 and d == 128 also an fp32 dQ accumulator of
+ * (N padded) * H * d floats. Returns 0 for an invalid shape. */
+ULY_API size_t ulysses_attn_bwd_workspace_size(int64_t N, int P, int H, int H_kv, int d, int deterministic);
 
 /* Attention backward on the head shards of ranks [rank_lo, rank_hi). The pages
  * train through the layer but do not write its backward; this is the gradient
@@ -149,15 +150,22 @@ ULY_API size_t ulysses_attn_bwd_workspace_size(int64_t N, int P, int H, int H_kv
  * o, do_head (head shards, as in the forward) and lse_head from the forward.
  * Outputs dq_head (H/P heads), dk_head, dv_head (H_kv/P heads), bf16.
  * workspace: caller-owned device memory of at least
- * ulysses_attn_bwd_workspace_size() bytes, 256-byte aligned; its contents on
- * entry do not matter. */
+ * ulysses_attn_bwd_workspace_size() bytes (same `deterministic`), 256-byte
+ * aligned; its contents on entry do not matter.
+ * deterministic != 0: two passes (K/V-stationary dK, dV; Q-stationary dQ) that
+ * recompute S and dP, no atomics: bit-identical results run to run.
+ * deterministic == 0 (d == 128): one pass computes dK, dV and dQ together and
+ * sums dQ in fp32 with vector reductions in L2 (about 5/7 of the tensor work);
+ * dK and dV are the same bits as the two-pass path, dQ agrees to fp32 rounding
+ * but its low bits may differ between runs. With d == 64 both settings run
+ * the two-pass kernels. */
 ULY_API uly_status ulysses_attn_bwd(
     const void* const* q_head, const void* const* k_head, const void* const* v_head,
     const void* const* o_head, const float* const* lse_head, const void* const* do_head,
     void* const* dq_head, void* const* dk_head, void* const* dv_head,
     int64_t N, int P, int H, int H_kv, int d,
     const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
-    float softmax_scale,
+    float softmax_scale, int deterministic,
     void* workspace, size_t workspace_bytes,
     int rank_lo, int rank_hi, cudaStream_t stream);
 
@@ -165,15 +173,16 @@ ULY_API uly_status ulysses_attn_bwd(
  * the head->seq all-to-all of dQ, dK, dV, reading Q, K, V, O, dO from the
  * sequence shards and writing dQ, dK, dV into them (all arrays: P sequence
  * shards; lse_head: per rank in range, from ulysses_attn_fwd_seq or
- * ulysses_attn_fwd). Workspace as ulysses_attn_bwd. Bit-identical to the
- * separate calls. Needs (N/P) % 128 == 0; otherwise ULY_ERR_UNSUPPORTED. */
+ * ulysses_attn_fwd). Workspace and `deterministic` as ulysses_attn_bwd;
+ * bit-identical to the separate calls (for dQ with deterministic == 0: up to
+ * the run-to-run order of the fp32 sums). Needs (N/P) % 128 == 0; otherwise ULY_ERR_UNSUPPORTED. */
 ULY_API uly_status ulysses_attn_bwd_seq(
     const void* const* q_seq, const void* const* k_seq, const void* const* v_seq,
     const void* const* o_seq, const float* const* lse_head, const void* const* do_seq,
     void* const* dq_seq, void* const* dk_seq, void* const* dv_seq,
     int64_t N, int P, int H, int H_kv, int d,
     const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
-    float softmax_scale,
+    float softmax_scale, int deterministic,
     void* workspace, size_t workspace_bytes,
     int rank_lo, int rank_hi, cudaStream_t stream);
 
@@ -181,12 +190,12 @@ ULY_API uly_status ulysses_attn_bwd_seq(
  * plugin or embedded runtime that hands this library only its input and output
  * buffers and owns every allocation itself, or a loop where cudaMalloc (which
  * can synchronise the device) is not allowed. The paper has no counterpart;
- * this is a deployment variant of ulysses_attn_bwd with identical arguments
- * and results, minus workspace/workspace_bytes.
+ * this is a deployment variant of ulysses_attn_bwd with deterministic = 1 and
+ * identical arguments and results, minus deterministic/workspace/workspace_bytes.
  *
  * Its scratch is a fixed 32 MiB device array inside this library (held by every
  * GPU that loads the library until the process exits); it needs
- * ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d) <= 32 MiB, i.e.
+ * ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, 1) <= 32 MiB, i.e.
  * H * (N rounded up to a multiple of 128) <= 4,194,304 (for example
  * N <= 131072 at H = 32); larger sizes return ULY_ERR_UNSUPPORTED with nothing
  * launched. It calls no allocator. The first call on each device looks up the

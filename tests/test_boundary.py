@@ -91,17 +91,28 @@ def test_a2a_validation(L):
 
 
 def test_bwd_validation_and_workspace_size(L):
-    ws = L.ulysses_attn_bwd_workspace_size(8192, 4, 32, 8, 128)
-    assert ws >= 2 * 4 * 8 * 8192 * 4          # lse*log2(e) and D_i per (rank, head, row)
-    assert L.ulysses_attn_bwd_workspace_size(8192, 3, 32, 8, 128) == 0     # invalid shape -> 0
+    ws = L.ulysses_attn_bwd_workspace_size(8192, 4, 32, 8, 128, 1)
+    assert ws == 2 * 4 * 8 * 8192 * 4          # lse*log2(e) and D_i per (rank, head, row)
+    # one pass (d = 128): plus the fp32 dQ accumulator, N x H x d floats
+    assert L.ulysses_attn_bwd_workspace_size(8192, 4, 32, 8, 128, 0) == ws + 8192 * 32 * 128 * 4
+    # d = 64 always runs the two-pass kernels: no accumulator
+    assert L.ulysses_attn_bwd_workspace_size(8192, 4, 32, 8, 64, 0) == ws
+    # rows are padded to a multiple of 128
+    assert L.ulysses_attn_bwd_workspace_size(200, 2, 8, 8, 128, 0) == 2 * 2 * 4 * 256 * 4 + 256 * 8 * 128 * 4
+    assert L.ulysses_attn_bwd_workspace_size(8192, 3, 32, 8, 128, 0) == 0     # invalid shape -> 0
     P = 2
     p = _arr([GOOD] * P)
-    # workspace too small / misaligned
-    assert L.ulysses_attn_bwd(p, p, p, p, p, p, p, p, p, 256, P, 8, 8, 64, None, 0, 0, 0.0,
-                              ctypes.c_void_p(GOOD), 16, 0, P, None) == 1
-    need = L.ulysses_attn_bwd_workspace_size(256, P, 8, 8, 64)
-    assert L.ulysses_attn_bwd(p, p, p, p, p, p, p, p, p, 256, P, 8, 8, 64, None, 0, 0, 0.0,
-                              ctypes.c_void_p(GOOD + 16), need, 0, P, None) == 1
+    for det in (0, 1):
+        # workspace too small / misaligned
+        assert L.ulysses_attn_bwd(p, p, p, p, p, p, p, p, p, 256, P, 8, 8, 128, None, 0, 0, 0.0, det,
+                                  ctypes.c_void_p(GOOD), 16, 0, P, None) == 1
+        need = L.ulysses_attn_bwd_workspace_size(256, P, 8, 8, 128, det)
+        assert L.ulysses_attn_bwd(p, p, p, p, p, p, p, p, p, 256, P, 8, 8, 128, None, 0, 0, 0.0, det,
+                                  ctypes.c_void_p(GOOD + 16), need, 0, P, None) == 1
+    # a workspace sized for the two-pass path is too small for the one-pass path
+    need1 = L.ulysses_attn_bwd_workspace_size(256, P, 8, 8, 128, 1)
+    assert L.ulysses_attn_bwd(p, p, p, p, p, p, p, p, p, 256, P, 8, 8, 128, None, 0, 0, 0.0, 0,
+                              ctypes.c_void_p(GOOD), need1, 0, P, None) == 1
 
 
 def test_fused_entry_points_need_shards_of_128_tokens(L):
@@ -109,7 +120,7 @@ def test_fused_entry_points_need_shards_of_128_tokens(L):
     p = _arr([GOOD] * P)
     # N/P = 100: a 128-token tile would straddle two shards
     assert L.ulysses_attn_fwd_seq(p, p, p, p, p, 200, P, 8, 8, 64, None, 0, 0, 0.0, 1, 0, P, None) == 2
-    assert L.ulysses_attn_bwd_seq(p, p, p, p, p, p, p, p, p, 200, P, 8, 8, 64, None, 0, 0, 0.0,
+    assert L.ulysses_attn_bwd_seq(p, p, p, p, p, p, p, p, p, 200, P, 8, 8, 64, None, 0, 0, 0.0, 1,
                                   ctypes.c_void_p(GOOD), 1 << 20, 0, P, None) == 2
     # every sequence shard must be given, even for a partial rank range
     half = _arr([GOOD, 0])

@@ -1,8 +1,10 @@
 """The fused layer (the all-to-alls folded into the attention kernels'
 addressing: ulysses_attn_fwd_seq / ulysses_attn_bwd_seq) against the three-call
-path it replaces: bit-identical O, LSE, dQ, dK, dV, since the kernels do the
-same arithmetic in the same order and only fetch and store elsewhere. One case
-is also checked against the fp64 oracle directly."""
+path it replaces: bit-identical O, LSE, dQ, dK, dV with the two-pass backward,
+since the kernels do the same arithmetic in the same order and only fetch and
+store elsewhere; with the one-pass backward everything but dQ (whose fp32 sums
+run in timing-dependent order). One case is also checked against the fp64
+oracle directly."""
 import numpy as np
 import pytest
 import torch
@@ -20,12 +22,12 @@ def _draw(N, H, H_kv, d, seed):
     return mk((N, H, d)), mk((N, H_kv, d)), mk((N, H_kv, d)), mk((N, H, d))
 
 
-def _run(q, k, v, do, P, cu, fused):
+def _run(q, k, v, do, P, cu, fused, deterministic=False):
     import ulysses_sequence_parallelism_b200 as U
     N, H, d = q.shape
     H_kv = k.shape[1]
     cu_t = None if cu is None else torch.tensor(np.asarray(cu, np.int32), device="cuda")
-    layer = U.UlyssesLayer(N, P, H, H_kv, d, cu_seqlens=cu_t, fused=fused)
+    layer = U.UlyssesLayer(N, P, H, H_kv, d, cu_seqlens=cu_t, fused=fused, deterministic=deterministic)
     o = layer.forward(shards_to_dev(q, P), shards_to_dev(k, P), shards_to_dev(v, P))
     g = layer.backward(shards_to_dev(do, P))
     torch.cuda.synchronize()
@@ -44,13 +46,20 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("deterministic", [True, False], ids=["twopass", "onepass"])
 @pytest.mark.parametrize("N,P,H,H_kv,d,cu", CASES)
-def test_fused_layer_is_bit_identical_to_three_calls(N, P, H, H_kv, d, cu):
+def test_fused_layer_is_bit_identical_to_three_calls(N, P, H, H_kv, d, cu, deterministic):
     q, k, v, do = _draw(N, H, H_kv, d, seed=N + P + d)
-    a = _run(q, k, v, do, P, cu, fused=False)
-    b = _run(q, k, v, do, P, cu, fused=True)
+    a = _run(q, k, v, do, P, cu, fused=False, deterministic=deterministic)
+    b = _run(q, k, v, do, P, cu, fused=True, deterministic=deterministic)
     for n in ("o", "lse", "dq", "dk", "dv"):
-        assert np.array_equal(a[n], b[n]), n
+        if n == "dq" and not deterministic and d == 128:
+            wa = a[n].view(np.uint16).astype(np.uint32) << 16
+            wb = b[n].view(np.uint16).astype(np.uint32) << 16
+            fa, fb = wa.view(np.float32).astype(np.float64), wb.view(np.float32).astype(np.float64)
+            assert np.all(np.abs(fa - fb) <= np.abs(fa) * 2.0 ** -7 + 1e-5 * np.abs(fa).max()), n
+        else:
+            assert np.array_equal(a[n], b[n]), n
 
 
 def test_fused_layer_matches_oracle():

@@ -43,7 +43,7 @@ def test_noalloc_backward_matches_workspace_backward_twice():
         U.ulysses_a2a_seq_to_head(do, None, None, layer.do_h, None, None, N, P, H, H_kv, d)
         # reference: the entry point that takes a caller-owned workspace
         U.ulysses_attn_bwd(layer.q_h, layer.k_h, layer.v_h, layer.o_h, layer.lse, layer.do_h, layer.dq_h,
-                           layer.dk_h, layer.dv_h, N, P, H, H_kv, d, layer.workspace, cu)
+                           layer.dk_h, layer.dv_h, N, P, H, H_kv, d, layer.workspace, cu, deterministic=True)
         ref = [f64(torch.cat(x, 0)) for x in (layer.dq_h, layer.dk_h, layer.dv_h)]
         dq = [torch.full_like(x, float("nan")) for x in layer.dq_h]
         dk = [torch.full_like(x, float("nan")) for x in layer.dk_h]

@@ -34,9 +34,9 @@ _SIGS = {
     "ulysses_a2a_head_to_seq": [_vpp, _vpp, _vpp, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _v, _i, _i, _i, _v],
     "ulysses_attn_fwd": [_vpp, _vpp, _vpp, _vpp, _fpp, _i64, _i, _i, _i, _i, _v, _i, _i, ctypes.c_float, _i,
                          _i, _i, _v],
-    "ulysses_attn_bwd_workspace_size": [_i64, _i, _i, _i, _i],
+    "ulysses_attn_bwd_workspace_size": [_i64, _i, _i, _i, _i, _i],
     "ulysses_attn_bwd": [_vpp, _vpp, _vpp, _vpp, _fpp, _vpp, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _v, _i, _i,
-                         ctypes.c_float, _v, ctypes.c_size_t, _i, _i, _v],
+                         ctypes.c_float, _i, _v, ctypes.c_size_t, _i, _i, _v],
     "ulysses_status_string": [_i],
     "ulysses_get_device_status": [_v, ctypes.POINTER(ctypes.c_uint32)],
     "ulysses_set_wait_limit": [ctypes.c_uint32],
@@ -44,7 +44,7 @@ _SIGS = {
     "ulysses_attn_fwd_seq": [_vpp, _vpp, _vpp, _vpp, _fpp, _i64, _i, _i, _i, _i, _v, _i, _i, ctypes.c_float, _i,
                              _i, _i, _v],
     "ulysses_attn_bwd_seq": [_vpp, _vpp, _vpp, _vpp, _fpp, _vpp, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _v, _i,
-                             _i, ctypes.c_float, _v, ctypes.c_size_t, _i, _i, _v],
+                             _i, ctypes.c_float, _i, _v, ctypes.c_size_t, _i, _i, _v],
     "ulysses_attn_bwd_noalloc": [_vpp, _vpp, _vpp, _vpp, _fpp, _vpp, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _v, _i,
                                  _i, ctypes.c_float, _i, _i, _v],
 }

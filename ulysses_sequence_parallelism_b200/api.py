@@ -94,32 +94,35 @@ def ulysses_attn_fwd_seq(q_seq, k_seq, v_seq, o_seq, lse_head, N, P, H, H_kv, d,
 
 def ulysses_attn_bwd_seq(q_seq, k_seq, v_seq, o_seq, lse_head, do_seq, dq_seq, dk_seq, dv_seq, N, P, H, H_kv, d,
                          workspace: torch.Tensor, cu_seqlens=None, max_seqlen=0, softmax_scale=0.0, rank_lo=0,
-                         rank_hi=None, stream=None):
+                         rank_hi=None, stream=None, deterministic=False):
     cu, ns = _cu(cu_seqlens)
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     code = lib().ulysses_attn_bwd_seq(
         _ptrs(q_seq, P), _ptrs(k_seq, P), _ptrs(v_seq, P), _ptrs(o_seq, P), _ptrs(lse_head, P, torch.float32),
         _ptrs(do_seq, P), _ptrs(dq_seq, P), _ptrs(dk_seq, P), _ptrs(dv_seq, P), N, P, H, H_kv, d, cu, ns,
-        max_seqlen, float(softmax_scale), ctypes.c_void_p(workspace.data_ptr()),
+        max_seqlen, float(softmax_scale), int(bool(deterministic)), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), rank_lo, P if rank_hi is None else rank_hi, _stream(stream))
     check("ulysses_attn_bwd_seq", code)
 
 
-def ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d) -> int:
-    return int(lib().ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d))
+def ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, deterministic=False) -> int:
+    return int(lib().ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, int(bool(deterministic))))
 
 
 def ulysses_attn_bwd(q_head, k_head, v_head, o_head, lse_head, do_head, dq_head, dk_head, dv_head, N, P, H,
                      H_kv, d, workspace: torch.Tensor, cu_seqlens=None, max_seqlen=0, softmax_scale=0.0,
-                     rank_lo=0, rank_hi=None, stream=None):
+                     rank_lo=0, rank_hi=None, stream=None, deterministic=False):
+    """deterministic=False (d=128): one-pass backward, dQ summed in fp32 by L2
+    reductions (run-to-run low-bit differences in dQ). True: two-pass,
+    bit-reproducible. The workspace must be sized with the same setting."""
     cu, ns = _cu(cu_seqlens)
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     code = lib().ulysses_attn_bwd(
         _ptrs(q_head, P), _ptrs(k_head, P), _ptrs(v_head, P), _ptrs(o_head, P), _ptrs(lse_head, P, torch.float32),
         _ptrs(do_head, P), _ptrs(dq_head, P), _ptrs(dk_head, P), _ptrs(dv_head, P), N, P, H, H_kv, d, cu, ns,
-        max_seqlen, float(softmax_scale), ctypes.c_void_p(workspace.data_ptr()),
+        max_seqlen, float(softmax_scale), int(bool(deterministic)), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), rank_lo, P if rank_hi is None else rank_hi, _stream(stream))
     check("ulysses_attn_bwd", code)
 
@@ -150,7 +153,7 @@ class UlyssesLayer:
 
     def __init__(self, N: int, P: int, H: int, H_kv: int, d: int, device="cuda", cu_seqlens=None,
                  max_seqlen: int = 0, softmax_scale: float = 0.0, backward: bool = True,
-                 rank_sequential: bool = False, fused: bool = False):
+                 rank_sequential: bool = False, fused: bool = False, deterministic: bool = False):
         if P > MAX_RANKS:
             raise ValueError(f"P <= {MAX_RANKS}")
         self.N, self.P, self.H, self.H_kv, self.d = N, P, H, H_kv, d
@@ -158,6 +161,8 @@ class UlyssesLayer:
         self.max_seqlen = max_seqlen
         self.scale = softmax_scale
         self.rank_sequential = rank_sequential
+        # deterministic: two-pass backward with bit-reproducible dQ (else one pass)
+        self.deterministic = deterministic
         # fused: the all-to-alls happen inside the attention kernels' addressing
         # (ulysses_attn_fwd_seq / ulysses_attn_bwd_seq); no head-sharded copies.
         self.fused = fused
@@ -173,7 +178,7 @@ class UlyssesLayer:
         self.backward_enabled = backward and not rank_sequential
         if self.backward_enabled:
             self.do_h, self.dq_h, self.dk_h, self.dv_h = mk(H), mk(H), mk(H_kv), mk(H_kv)
-            ws = ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d)
+            ws = ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, deterministic)
             self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
 
     def _rank_bufs(self, bufs, r):
@@ -216,10 +221,12 @@ class UlyssesLayer:
         if self.fused:
             q_seq, k_seq, v_seq, o_seq = self._seq_in
             ulysses_attn_bwd_seq(q_seq, k_seq, v_seq, o_seq, self.lse, do_seq, dq_seq, dk_seq, dv_seq, N, P, H,
-                                 H_kv, d, self.workspace, self.cu, self.max_seqlen, self.scale)
+                                 H_kv, d, self.workspace, self.cu, self.max_seqlen, self.scale,
+                                 deterministic=self.deterministic)
             return dq_seq, dk_seq, dv_seq
         ulysses_a2a_seq_to_head(do_seq, None, None, self.do_h, None, None, N, P, H, H_kv, d, self.cu)
         ulysses_attn_bwd(self.q_h, self.k_h, self.v_h, self.o_h, self.lse, self.do_h, self.dq_h, self.dk_h,
-                         self.dv_h, N, P, H, H_kv, d, self.workspace, self.cu, self.max_seqlen, self.scale)
+                         self.dv_h, N, P, H, H_kv, d, self.workspace, self.cu, self.max_seqlen, self.scale,
+                         deterministic=self.deterministic)
         ulysses_a2a_head_to_seq(self.dq_h, self.dk_h, self.dv_h, dq_seq, dk_seq, dv_seq, N, P, H, H_kv, d, self.cu)
         return dq_seq, dk_seq, dv_seq

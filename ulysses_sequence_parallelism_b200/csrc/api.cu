@@ -124,17 +124,17 @@ uly_status ulysses_attn_fwd(const void* const* q_head, const void* const* k_head
   return from_cuda(uly::launch_attn_fwd(s, q_head, k_head, v_head, o_head, lse_head, stream));
 }
 
-size_t ulysses_attn_bwd_workspace_size(int64_t N, int P, int H, int H_kv, int d) {
+size_t ulysses_attn_bwd_workspace_size(int64_t N, int P, int H, int H_kv, int d, int deterministic) {
   if (check_shape(N, P, H, H_kv, d, 0, P > 0 ? P : 1) != ULY_OK) return 0;
-  return uly::attn_bwd_workspace_bytes(N, P, H / P, d);
+  return uly::attn_bwd_workspace_bytes(N, P, H / P, d, deterministic);
 }
 
 uly_status ulysses_attn_bwd(const void* const* q_head, const void* const* k_head, const void* const* v_head,
                             const void* const* o_head, const float* const* lse_head, const void* const* do_head,
                             void* const* dq_head, void* const* dk_head, void* const* dv_head, int64_t N, int P,
                             int H, int H_kv, int d, const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
-                            float softmax_scale, void* workspace, size_t workspace_bytes, int rank_lo,
-                            int rank_hi, cudaStream_t stream) {
+                            float softmax_scale, int deterministic, void* workspace, size_t workspace_bytes,
+                            int rank_lo, int rank_hi, cudaStream_t stream) {
   (void)max_seqlen;
   uly_status st = check_shape(N, P, H, H_kv, d, rank_lo, rank_hi);
   if (st != ULY_OK) return st;
@@ -147,11 +147,11 @@ uly_status ulysses_attn_bwd(const void* const* q_head, const void* const* k_head
       !ranks_ok(cv(dk_head), rank_lo, rank_hi) || !ranks_ok(cv(dv_head), rank_lo, rank_hi))
     return ULY_ERR_INVALID_ARG;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ULY_ERR_INVALID_ARG;
-  if (workspace_bytes < uly::attn_bwd_workspace_bytes(N, P, H / P, d)) return ULY_ERR_INVALID_ARG;
+  if (workspace_bytes < uly::attn_bwd_workspace_bytes(N, P, H / P, d, deterministic)) return ULY_ERR_INVALID_ARG;
   uly::AttnShape s{static_cast<int>(N), P, H / P, H_kv / P, d, cu_seqlens, cu_seqlens ? num_seqs : 1,
                    resolve_scale(softmax_scale, d), rank_lo, rank_hi};
   return from_cuda(uly::launch_attn_bwd(s, q_head, k_head, v_head, o_head, lse_head, do_head, dq_head, dk_head,
-                                        dv_head, workspace, stream));
+                                        dv_head, workspace, deterministic, stream));
 }
 
 uly_status ulysses_attn_fwd_seq(const void* const* q_seq, const void* const* k_seq, const void* const* v_seq,
@@ -176,8 +176,8 @@ uly_status ulysses_attn_bwd_seq(const void* const* q_seq, const void* const* k_s
                                 const void* const* o_seq, const float* const* lse_head, const void* const* do_seq,
                                 void* const* dq_seq, void* const* dk_seq, void* const* dv_seq, int64_t N, int P,
                                 int H, int H_kv, int d, const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
-                                float softmax_scale, void* workspace, size_t workspace_bytes, int rank_lo,
-                                int rank_hi, cudaStream_t stream) {
+                                float softmax_scale, int deterministic, void* workspace,
+                                size_t workspace_bytes, int rank_lo, int rank_hi, cudaStream_t stream) {
   (void)max_seqlen;
   uly_status st = check_shape(N, P, H, H_kv, d, rank_lo, rank_hi);
   if (st != ULY_OK) return st;
@@ -190,11 +190,11 @@ uly_status ulysses_attn_bwd_seq(const void* const* q_seq, const void* const* k_s
       !ranks_ok(reinterpret_cast<const void* const*>(lse_head), rank_lo, rank_hi))
     return ULY_ERR_INVALID_ARG;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ULY_ERR_INVALID_ARG;
-  if (workspace_bytes < uly::attn_bwd_workspace_bytes(N, P, H / P, d)) return ULY_ERR_INVALID_ARG;
+  if (workspace_bytes < uly::attn_bwd_workspace_bytes(N, P, H / P, d, deterministic)) return ULY_ERR_INVALID_ARG;
   uly::AttnShape s{static_cast<int>(N), P, H / P, H_kv / P, d, cu_seqlens, cu_seqlens ? num_seqs : 1,
                    resolve_scale(softmax_scale, d), rank_lo, rank_hi};
   return from_cuda(uly::launch_attn_bwd_seq(s, q_seq, k_seq, v_seq, o_seq, lse_head, do_seq, dq_seq, dk_seq,
-                                            dv_seq, workspace, stream));
+                                            dv_seq, workspace, deterministic, stream));
 }
 
 const char* ulysses_status_string(uly_status s) {

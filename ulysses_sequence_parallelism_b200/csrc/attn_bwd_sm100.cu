@@ -8,7 +8,7 @@
 //   dK_j = scale sum_i dS_ij q_i,   dQ_i = scale sum_j dS_ij k_j
 // dK/dV of a key/value head are summed over the H/H_kv query heads reading it.
 //
-// Three launches, deterministic (no atomics anywhere):
+// With deterministic == 1 (or head dim 64): three launches, no atomics anywhere:
 //  1. prep : D_i and lse_i*log2(e) per (rank, head, row) into a workspace
 //            padded to a multiple of 128 rows (padding: lse = +inf, D = 0, so
 //            padded rows contribute exactly zero).
@@ -24,6 +24,9 @@
 //              the two warpgroups on the two key halves); dQ += dS K (TS MMA).
 // S and dP are recomputed in (3): 7 block GEMMs instead of 5, in exchange for
 // no fp32 atomics, no dQ accumulator traffic and a bit-reproducible result.
+// With deterministic == 0 and head dim 128, the one-pass kernel
+// (attn_bwd_onepass_sm100.cuh) replaces (2) and (3): 5 block GEMMs, dQ summed
+// in fp32 by L2 vector reductions into a workspace accumulator.
 // Layouts: as in the forward, seq == 0 reads and writes rank r's head shards
 // ([N, Hx/P, d]); seq == 1 (the fused path) maps the sequence shards
 // ([N/P, Hx, d], N/P a multiple of 128) and addresses rank r's heads as the
@@ -129,6 +132,7 @@ struct DkdvArgs {
   RankPtrsMut dk, dv;
   const float* lse2;
   const float* Dv;
+  float* dqacc;                 // one-pass kernel only: fp32 dQ accumulator
   const int32_t* cu;
   int num_seqs;
   int N, Npad, Hl, Hkvl, group;
@@ -708,6 +712,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_kernel(const __grid_c
   }
 }
 
+}  // namespace bwd_sm100
+}  // namespace uly
+
+#include "attn_bwd_onepass_sm100.cuh"
+
+namespace uly {
+namespace bwd_sm100 {
+
 // ====================================================================== host
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -767,18 +779,67 @@ cudaError_t launch_all(const AttnShape& s, const PrepArgs& pa, const DkdvArgs& k
   }
 }
 
+// prep, zero the dQ accumulator of the ranks in range, one-pass dK/dV/dQ, dQ conversion
+cudaError_t launch_onepass(const AttnShape& s, const PrepArgs& pa, const DkdvArgs& ka, const RankPtrsMut& dq,
+                           cudaStream_t stream) {
+  constexpr int D = onepass::D;
+  const int nranks = s.rank_hi - s.rank_lo;
+  {
+    constexpr int RPB = 256 / (D / 8);
+    const int64_t rows = static_cast<int64_t>(pa.Npad) * s.Hl * nranks;
+    bwd_prep_kernel<D><<<static_cast<unsigned>((rows + RPB - 1) / RPB), 256, 0, stream>>>(pa);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const size_t per_rank = static_cast<size_t>(s.Hl) * pa.Npad * D;   // floats
+  {
+    cudaError_t e = cudaMemsetAsync(ka.dqacc + per_rank * s.rank_lo, 0, per_rank * nranks * sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+  }
+  {
+    cudaError_t e = cudaFuncSetAttribute(onepass::attn_bwd_onepass_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, onepass::Layout::kAlloc);
+    if (e != cudaSuccess) return e;
+    dim3 grid(s.Hkvl * nranks, (s.N + TB - 1) / TB);
+    onepass::attn_bwd_onepass_kernel<<<grid, kThreads, onepass::Layout::kAlloc, stream>>>(ka);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  {
+    onepass::ConvArgs ca;
+    memset(&ca, 0, sizeof(ca));
+    ca.acc = ka.dqacc;
+    ca.dq = dq;
+    ca.N = s.N;
+    ca.Npad = pa.Npad;
+    ca.Hl = s.Hl;
+    ca.rank_lo = s.rank_lo;
+    ca.nranks = nranks;
+    ca.scale = s.scale;
+    ca.seq = pa.seq;
+    ca.n_loc = pa.n_loc;
+    ca.P = s.P;
+    const int64_t threads = static_cast<int64_t>(nranks) * s.Hl * (pa.Npad / 4) * 32;
+    onepass::dq_convert_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(ca);
+    return cudaGetLastError();
+  }
+}
+
 }  // namespace bwd_sm100
 
-size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d) {
-  (void)d;
+bool attn_bwd_onepass(int d, int deterministic) { return !deterministic && d == bwd_sm100::onepass::D; }
+
+size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d, int deterministic) {
   const int64_t npad = (N + bwd_sm100::TB - 1) / bwd_sm100::TB * bwd_sm100::TB;
-  return 2 * static_cast<size_t>(P) * Hl * npad * sizeof(float);
+  size_t bytes = 2 * static_cast<size_t>(P) * Hl * npad * sizeof(float);
+  if (attn_bwd_onepass(d, deterministic)) bytes += static_cast<size_t>(P) * Hl * npad * d * sizeof(float);
+  return bytes;
 }
 
 namespace bwd_sm100 {
 // Fills everything but the per-buffer pointers and tensor maps, then launches.
 cudaError_t launch_common(const AttnShape& s, PrepArgs& pa, DkdvArgs& ka, DqArgs& qa, void* workspace, int seq,
-                          cudaStream_t stream) {
+                          int deterministic, cudaStream_t stream) {
   const int Npad = padded_rows(s.N);
   float* lse2 = static_cast<float*>(workspace);
   float* Dv = lse2 + static_cast<size_t>(s.P) * s.Hl * Npad;
@@ -805,13 +866,18 @@ cudaError_t launch_common(const AttnShape& s, PrepArgs& pa, DkdvArgs& ka, DqArgs
   ka.scale_log2 = qa.scale_log2 = s.scale * kLog2e;
   ka.rank_lo = qa.rank_lo = s.rank_lo;
   qa.num_m_tiles = (s.N + TB - 1) / TB;
+  if (attn_bwd_onepass(s.d, deterministic)) {
+    ka.dqacc = Dv + static_cast<size_t>(s.P) * s.Hl * Npad;   // 512-byte aligned: Npad is a multiple of 128
+    return launch_onepass(s, pa, ka, qa.dq, stream);
+  }
   return s.d == 64 ? launch_all<64>(s, pa, ka, qa, stream) : launch_all<128>(s, pa, ka, qa, stream);
 }
 }  // namespace bwd_sm100
 
 cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void* const* k, const void* const* v,
                             const void* const* o, const float* const* lse, const void* const* dO, void* const* dq,
-                            void* const* dk, void* const* dv, void* workspace, cudaStream_t stream) {
+                            void* const* dk, void* const* dv, void* workspace, int deterministic,
+                            cudaStream_t stream) {
   using namespace bwd_sm100;
   EncodeTiledFn enc = get_encode();
   if (enc == nullptr) return cudaErrorNotSupported;
@@ -835,13 +901,13 @@ cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void
     ka.dv.p[r] = dv[r];
     qa.dq.p[r] = dq[r];
   }
-  return launch_common(s, pa, ka, qa, workspace, 0, stream);
+  return launch_common(s, pa, ka, qa, workspace, 0, deterministic, stream);
 }
 
 cudaError_t launch_attn_bwd_seq(const AttnShape& s, const void* const* q_seq, const void* const* k_seq,
                                 const void* const* v_seq, const void* const* o_seq, const float* const* lse,
                                 const void* const* do_seq, void* const* dq_seq, void* const* dk_seq,
-                                void* const* dv_seq, void* workspace, cudaStream_t stream) {
+                                void* const* dv_seq, void* workspace, int deterministic, cudaStream_t stream) {
   using namespace bwd_sm100;
   EncodeTiledFn enc = get_encode();
   if (enc == nullptr) return cudaErrorNotSupported;
@@ -866,7 +932,7 @@ cudaError_t launch_attn_bwd_seq(const AttnShape& s, const void* const* q_seq, co
     qa.dq.p[p] = dq_seq[p];
   }
   for (int r = s.rank_lo; r < s.rank_hi; ++r) pa.lse.p[r] = lse[r];
-  return launch_common(s, pa, ka, qa, workspace, 1, stream);
+  return launch_common(s, pa, ka, qa, workspace, 1, deterministic, stream);
 }
 
 }  // namespace uly

@@ -44,12 +44,12 @@ extern "C" uly_status ulysses_attn_bwd_noalloc(
     const float* const* lse_head, const void* const* do_head, void* const* dq_head, void* const* dk_head,
     void* const* dv_head, int64_t N, int P, int H, int H_kv, int d, const int32_t* cu_seqlens, int num_seqs,
     int max_seqlen, float softmax_scale, int rank_lo, int rank_hi, cudaStream_t stream) {
-  const size_t need = ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d);
+  const size_t need = ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, 1);
   if (need == 0) return ULY_ERR_INVALID_ARG;                        // invalid shape
   if (need > uly::noalloc::kScratchBytes) return ULY_ERR_UNSUPPORTED;  // beyond the fixed scratch
   void* scratch = nullptr;
   if (uly::noalloc::scratch_address(&scratch) != cudaSuccess) return ULY_ERR_CUDA;
   return ulysses_attn_bwd(q_head, k_head, v_head, o_head, lse_head, do_head, dq_head, dk_head, dv_head, N, P, H,
-                          H_kv, d, cu_seqlens, num_seqs, max_seqlen, softmax_scale, scratch,
+                          H_kv, d, cu_seqlens, num_seqs, max_seqlen, softmax_scale, 1, scratch,
                           uly::noalloc::kScratchBytes, rank_lo, rank_hi, stream);
 }

@@ -31,12 +31,14 @@ cudaError_t launch_attn_fwd_seq(const AttnShape& s, const void* const* q_seq, co
 cudaError_t launch_attn_bwd_seq(const AttnShape& s, const void* const* q_seq, const void* const* k_seq,
                                 const void* const* v_seq, const void* const* o_seq, const float* const* lse,
                                 const void* const* do_seq, void* const* dq_seq, void* const* dk_seq,
-                                void* const* dv_seq, void* workspace, cudaStream_t stream);
+                                void* const* dv_seq, void* workspace, int deterministic, cudaStream_t stream);
 
-size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d);
+// deterministic == 0 with d == 128 selects the one-pass backward (fp32 dQ
+// accumulator in the workspace); everything else runs the two-pass kernels.
+size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d, int deterministic);
 cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void* const* k,
                             const void* const* v, const void* const* o, const float* const* lse,
                             const void* const* dO, void* const* dq, void* const* dk, void* const* dv,
-                            void* workspace, cudaStream_t stream);
+                            void* workspace, int deterministic, cudaStream_t stream);
 
 }  // namespace uly
