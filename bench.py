@@ -42,6 +42,35 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def kernel_source_hash():
+    """sha256 over the kernel sources (name + bytes), to tell whether stored
+    ncu counters still describe the kernels being run."""
+    import glob
+    import hashlib
+    csrc = os.path.join(ROOT, "ulysses_sequence_parallelism_b200", "csrc")
+    files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
+                   glob.glob(os.path.join(csrc, "*.h")))
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def stored_traffic(workload, stage):
+    """DRAM bytes per call of `stage` from profiles/roofline_traffic.json, or
+    None when they were taken on other kernel sources or another workload."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "roofline_traffic.json")) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    if t.get("workload") != workload or t.get("source_sha256") != kernel_source_hash():
+        return None
+    return t.get(stage, {}).get("bytes")
+
+
 def flops(w, cu):
     pairs = workloads.causal_pairs(w.N, cu)
     return 4.0 * w.d * w.H * pairs, 10.0 * w.d * w.H * pairs, pairs
@@ -343,8 +372,9 @@ def main():
     if dom in ("attn_fwd", "attn_bwd"):
         achieved = (f_fwd if dom == "attn_fwd" else f_bwd) / (mean[dom] / 1e3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
-                "frac": achieved / tensor_peak, "traffic": None,
-                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)"}
+                "frac": achieved / tensor_peak, "traffic": stored_traffic(w.name if args.tokens is None else None, dom),
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                "traffic_source": "ncu DRAM bytes per call, profiles/roofline_traffic.json (null if the kernels changed)"}
     else:
         achieved = pb[dom] / (mean[dom] / 1e3) / 1e9
         hp = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -383,45 +413,42 @@ def main():
         del lf
 
     # ---------------------------------------------------------------- end to end through the public API
+    # HostPipeline: every step copies its inputs from pinned host memory and
+    # reads its results back; copies of neighbouring steps overlap the kernels.
     e2e = None
     if not args.no_e2e:
         pin = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
         n = N // P
-        hq = [pin(inp["q"][p * n:(p + 1) * n]) for p in range(P)]
-        hk = [pin(inp["k"][p * n:(p + 1) * n]) for p in range(P)]
-        hv = [pin(inp["v"][p * n:(p + 1) * n]) for p in range(P)]
-        hdo = [pin(inp["do"][p * n:(p + 1) * n]) for p in range(P)] if w.backward else []
-        outs_h = [torch.empty_like(x).pin_memory() for x in hq]
+        rows = lambda a: [pin(a[p * n:(p + 1) * n]) for p in range(P)]
+        host_in = {"q": rows(inp["q"]), "k": rows(inp["k"]), "v": rows(inp["v"])}
         if w.backward:
-            outs_h += [torch.empty_like(x).pin_memory() for x in hq + hk + hv]
-        dev_in = q + k + v + (do if w.backward else [])
-        host_in = hq + hk + hv + hdo
-        dev_out = o + ((dq + dk + dv) if w.backward else [])
-        h2d = sum(x.numel() * 2 for x in host_in)
-        d2h = sum(x.numel() * 2 for x in outs_h)
-
-        def e2e_step():
-            for hsrc, dd in zip(host_in, dev_in):
-                dd.copy_(hsrc, non_blocking=True)
-            layer.forward(q, k, v, o)
+            host_in["do"] = rows(inp["do"])
+        empty_like_pinned = lambda xs: [torch.empty_like(x).pin_memory() for x in xs]
+        host_out = []
+        for _ in range(2):
+            ho = {"o": empty_like_pinned(host_in["q"])}
             if w.backward:
-                layer.backward(do, dq, dk, dv)
-            for dsrc, hh in zip(dev_out, outs_h):
-                hh.copy_(dsrc, non_blocking=True)
-
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
-        torch.cuda.synchronize()
+                ho.update(dq=empty_like_pinned(host_in["q"]), dk=empty_like_pinned(host_in["k"]),
+                          dv=empty_like_pinned(host_in["v"]))
+            host_out.append(ho)
+        h2d = sum(x.numel() * 2 for xs in host_in.values() for x in xs)
+        d2h = sum(x.numel() * 2 for xs in host_out[0].values() for x in xs)
+        hp = U.HostPipeline(layer, device=dev)
+        for i in range(max(1, args.warmup)):
+            hp.submit(host_in, host_out[i & 1])
+        hp.synchronize()
         barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        e_ms, e_val = aggregate_over_ranks(a.elapsed_time(b) / args.steps, N, world, reduce_max)
+        a = torch.cuda.Event(enable_timing=True)
+        a.record(hp.s_in)
+        last = None
+        for i in range(args.steps):
+            last = hp.submit(host_in, host_out[i & 1])
+        hp.synchronize()
+        e_ms, e_val = aggregate_over_ranks(a.elapsed_time(last) / args.steps, N, world, reduce_max)
         e2e = {"value": e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+               "api": "HostPipeline (copies of neighbouring steps overlap the kernels)"}
+        del hp
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

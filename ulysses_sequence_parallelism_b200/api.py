@@ -21,6 +21,7 @@ __all__ = [
     "ulysses_a2a_seq_to_head", "ulysses_a2a_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_bwd",
     "ulysses_attn_bwd_workspace_size", "ulysses_get_device_status", "ulysses_set_wait_limit",
     "ulysses_selftest_bounded_wait", "ulysses_attn_fwd_seq", "ulysses_attn_bwd_seq", "UlyssesLayer",
+    "HostPipeline",
 ]
 
 
@@ -230,3 +231,78 @@ class UlyssesLayer:
                          deterministic=self.deterministic)
         ulysses_a2a_head_to_seq(self.dq_h, self.dk_h, self.dv_h, dq_seq, dk_seq, dv_seq, N, P, H, H_kv, d, self.cu)
         return dq_seq, dk_seq, dv_seq
+
+
+class HostPipeline:
+    """Layer steps whose inputs and results live in pinned host memory.
+
+    ``submit(host_in, host_out)`` enqueues one training step of ``layer``
+    (forward + backward when the layer has backward buffers): the host->device
+    copy of the step's sequence shards (Q, K, V, dO), the layer's kernels, and
+    the device->host copy of its results (O, dQ, dK, dV). Copies in, compute
+    and copies out run on three streams with two device buffer sets, so the
+    copies of neighbouring steps overlap this step's kernels and PCIe moves
+    data in both directions at once. Results of a step are in ``host_out``
+    once ``synchronize()`` returns (or its ``done`` event has completed).
+
+    host_in:  {"q": [P tensors], "k": [...], "v": [...], "do": [...]}
+    host_out: {"o": [...], "dq": [...], "dk": [...], "dv": [...]}
+    (pinned CPU tensors shaped like the sequence shards; "do", "dq", "dk",
+    "dv" only with backward).
+    """
+
+    def __init__(self, layer: "UlyssesLayer", device="cuda"):
+        self.layer = layer
+        N, P, H, H_kv, d = layer.N, layer.P, layer.H, layer.H_kv, layer.d
+        bf = torch.bfloat16
+        n = N // P
+        shard = lambda hx: [torch.empty(n, hx, d, dtype=bf, device=device) for _ in range(P)]
+        self.bwd = layer.backward_enabled
+        self.ins = [{"q": shard(H), "k": shard(H_kv), "v": shard(H_kv), **({"do": shard(H)} if self.bwd else {})}
+                    for _ in range(2)]
+        self.outs = [{"o": shard(H), **({"dq": shard(H), "dk": shard(H_kv), "dv": shard(H_kv)} if self.bwd else {})}
+                     for _ in range(2)]
+        self.s_in = torch.cuda.Stream(device=device)
+        self.s_comp = torch.cuda.Stream(device=device)
+        self.s_out = torch.cuda.Stream(device=device)
+        self.in_free = [None, None]      # compute finished reading input set j
+        self.out_free = [None, None]     # copy-out finished reading output set j
+        self.k = 0
+
+    def submit(self, host_in, host_out):
+        j = self.k & 1
+        self.k += 1
+        dev_in, dev_out = self.ins[j], self.outs[j]
+        loaded = torch.cuda.Event()
+        with torch.cuda.stream(self.s_in):
+            if self.in_free[j] is not None:
+                self.s_in.wait_event(self.in_free[j])
+            for name, bufs in dev_in.items():
+                for dst, src in zip(bufs, host_in[name]):
+                    dst.copy_(src, non_blocking=True)
+            loaded.record(self.s_in)
+        computed, in_free = torch.cuda.Event(), torch.cuda.Event()
+        with torch.cuda.stream(self.s_comp):
+            self.s_comp.wait_event(loaded)
+            if self.out_free[j] is not None:
+                self.s_comp.wait_event(self.out_free[j])
+            L = self.layer
+            L.forward(dev_in["q"], dev_in["k"], dev_in["v"], dev_out["o"])
+            if self.bwd:
+                L.backward(dev_in["do"], dev_out["dq"], dev_out["dk"], dev_out["dv"])
+            in_free.record(self.s_comp)
+            computed.record(self.s_comp)
+        self.in_free[j] = in_free
+        done = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(computed)
+            for name, bufs in dev_out.items():
+                for dst, src in zip(host_out[name], bufs):
+                    dst.copy_(src, non_blocking=True)
+            done.record(self.s_out)
+        self.out_free[j] = done
+        return done
+
+    def synchronize(self):
+        for s in (self.s_in, self.s_comp, self.s_out):
+            s.synchronize()
