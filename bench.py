@@ -42,18 +42,15 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
-    """sha256 over the kernel sources (name + bytes), to tell whether stored
-    ncu counters still describe the kernels being run."""
-    import glob
+def kernel_source_hash(files):
+    """sha256 over the named kernel sources (name + bytes), to tell whether
+    stored ncu counters still describe the kernels being run."""
     import hashlib
     csrc = os.path.join(ROOT, "ulysses_sequence_parallelism_b200", "csrc")
-    files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
-                   glob.glob(os.path.join(csrc, "*.h")))
     h = hashlib.sha256()
     for f in files:
-        h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
+        h.update(f.encode())
+        with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
 
@@ -64,11 +61,12 @@ def stored_traffic(workload, stage):
     try:
         with open(os.path.join(ROOT, "profiles", "roofline_traffic.json")) as f:
             t = json.load(f)
+        st = t[stage]
+        if t.get("workload") != workload or st["source_sha256"] != kernel_source_hash(st["sources"]):
+            return None
+        return st["bytes"]
     except Exception:
         return None
-    if t.get("workload") != workload or t.get("source_sha256") != kernel_source_hash():
-        return None
-    return t.get(stage, {}).get("bytes")
 
 
 def flops(w, cu):
@@ -412,6 +410,41 @@ def main():
                  "note": "all-to-alls folded into the attention kernels' addressing (no permute launches)"}
         del lf
 
+    # ---------------------------------------------------------------- head fragmentation (NEXT-3)
+    # each rank processes its heads one GQA group at a time: same results, a
+    # fraction of the full-sequence activation buffers
+    frag = None
+    if w.backward:
+        g = H // H_kv
+        lfr = U.UlyssesLayer(N, P, H, H_kv, d, device=dev, cu_seqlens=cu, head_fragment=g,
+                             deterministic=args.deterministic)
+
+        def frag_step():
+            lfr.forward(q, k, v, o)
+            lfr.backward(do, dq, dk, dv)
+
+        for _ in range(max(1, min(args.warmup, 2))):
+            frag_step()
+        torch.cuda.synchronize()
+        barrier()
+        fa, fb_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_fr = max(1, min(args.steps, 5))
+        fa.record(stream)
+        for _ in range(n_fr):
+            frag_step()
+        fb_.record(stream)
+        torch.cuda.synchronize()
+        fr_ms, fr_val = aggregate_over_ranks(fa.elapsed_time(fb_) / n_fr, N, world, reduce_max)
+        nbytes = lambda ts: sum(t.numel() * t.element_size() for t in ts)
+        frag_bytes = nbytes([lfr.q_f, lfr.k_f, lfr.v_f, lfr.o_f, lfr.do_f, lfr.dq_f, lfr.dk_f, lfr.dv_f,
+                             lfr.workspace])
+        full_bytes = nbytes(layer.q_h + layer.k_h + layer.v_h + layer.o_h + layer.do_h + layer.dq_h + layer.dk_h +
+                            layer.dv_h + [layer.workspace])
+        frag = {"value": fr_val, "unit": "tokens/s", "ms_per_step": fr_ms, "steps": n_fr, "head_fragment": g,
+                "fragments_per_step": P * (H // P) // g, "head_side_bytes": frag_bytes,
+                "head_side_bytes_unfragmented": full_bytes}
+        del lfr
+
     # ---------------------------------------------------------------- end to end through the public API
     # HostPipeline: every step copies its inputs from pinned host memory and
     # reads its results back; copies of neighbouring steps overlap the kernels.
@@ -468,7 +501,7 @@ def main():
                        "parallelism": f"{P} virtual ranks per GPU; {world} independent replica(s)"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk, "detail": detail, "fused": fused,
+            "clocks": clk, "detail": detail, "fused": fused, "head_fragment": frag,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

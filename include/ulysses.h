@@ -96,6 +96,32 @@ ULY_API uly_status ulysses_a2a_head_to_seq(
     const int32_t* cu_seqlens, int num_seqs,
     int rank_lo, int rank_hi, cudaStream_t stream);
 
+/* Head fragments ("fragmentation by heads": q2bstudio.com, "Ulysses Unleashed:
+ * Context Parallelism with Fragmentation by Heads" -- a rank may process its
+ * heads a few at a time, one fragment after another, so that only one
+ * fragment's full-sequence activations exist at once).
+ * ulysses_a2a_seq_to_head_frag gathers global query heads
+ * [head_lo, head_lo + num_heads) of every token from the P sequence shards
+ * x0_seq ([N/P, H, d] each) into ONE buffer x0_frag [N, num_heads, d], and
+ * likewise their key/value heads [head_lo/g, (head_lo + num_heads)/g)
+ * (g = H/H_kv) from x1_seq/x2_seq ([N/P, H_kv, d]) into x1_frag/x2_frag
+ * [N, num_heads/g, d]; ulysses_a2a_head_to_seq_frag is the exact inverse and
+ * writes only the fragment's head columns of the sequence shards.
+ * The fragment must be whole GQA groups (head_lo and num_heads multiples of g)
+ * inside one rank's heads [r*H/P, (r+1)*H/P); else ULY_ERR_INVALID_ARG.
+ * Attention on a fragment is ulysses_attn_fwd / ulysses_attn_bwd with P = 1,
+ * H = num_heads, H_kv = num_heads/g on the fragment buffers (heads do not
+ * interact). x1/x2 may be NULL (both sides). Bit copies; all pointers 16-byte
+ * aligned; caller-owned; asynchronous on `stream`. */
+ULY_API uly_status ulysses_a2a_seq_to_head_frag(
+    const void* const* x0_seq, const void* const* x1_seq, const void* const* x2_seq,
+    void* x0_frag, void* x1_frag, void* x2_frag,
+    int64_t N, int P, int H, int H_kv, int d, int head_lo, int num_heads, cudaStream_t stream);
+ULY_API uly_status ulysses_a2a_head_to_seq_frag(
+    const void* x0_frag, const void* x1_frag, const void* x2_frag,
+    void* const* x0_seq, void* const* x1_seq, void* const* x2_seq,
+    int64_t N, int P, int H, int H_kv, int d, int head_lo, int num_heads, cudaStream_t stream);
+
 /* Causal (optionally packed-varlen) grouped-query flash attention forward on the
  * head shards of ranks [rank_lo, rank_hi): each rank runs attention by itself on
  * its heads, which do not interact (theaicatchup.com, ibid., citing DeepSpeed-Ulysses):

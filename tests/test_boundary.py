@@ -125,3 +125,28 @@ def test_fused_entry_points_need_shards_of_128_tokens(L):
     # every sequence shard must be given, even for a partial rank range
     half = _arr([GOOD, 0])
     assert L.ulysses_attn_fwd_seq(half, p, p, p, p, 256, P, 8, 8, 64, None, 0, 0, 0.0, 1, 0, 1, None) == 1
+
+
+def test_fragment_entry_points_validate_before_launch(L):
+    """Head fragments must be whole GQA groups inside one rank's heads; NULL
+    pairing of the k/v slots must match; anything else is rejected with
+    nothing launched (fake, never-dereferenced pointers)."""
+    P = 2
+    p = _arr([GOOD] * P)
+    f = ctypes.c_void_p(GOOD)
+    N, H, H_kv, d = 256, 8, 2, 128              # g = 4, 4 query heads per rank
+    ok_args = (N, P, H, H_kv, d)
+    # not whole groups
+    assert L.ulysses_a2a_seq_to_head_frag(p, p, p, f, f, f, *ok_args, 2, 4, None) == 1
+    assert L.ulysses_a2a_seq_to_head_frag(p, p, p, f, f, f, *ok_args, 0, 2, None) == 1
+    # crosses from rank 0's heads into rank 1's
+    assert L.ulysses_a2a_seq_to_head_frag(p, p, p, f, f, f, N, P, 8, 8, d, 2, 4, None) == 1
+    # out of range, empty
+    assert L.ulysses_a2a_seq_to_head_frag(p, p, p, f, f, f, *ok_args, 8, 4, None) == 1
+    assert L.ulysses_a2a_head_to_seq_frag(f, f, f, p, p, p, *ok_args, 0, 0, None) == 1
+    # k slot given on one side only; misaligned fragment pointer
+    assert L.ulysses_a2a_seq_to_head_frag(p, p, None, f, f, f, *ok_args, 0, 4, None) == 1
+    assert L.ulysses_a2a_head_to_seq_frag(ctypes.c_void_p(GOOD + 8), None, None, p, None, None, *ok_args, 4, 4,
+                                          None) == 1
+    # unsupported head dim
+    assert L.ulysses_a2a_seq_to_head_frag(p, None, None, f, None, None, N, P, H, H_kv, 96, 0, 4, None) == 2

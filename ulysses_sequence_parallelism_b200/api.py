@@ -21,7 +21,7 @@ __all__ = [
     "ulysses_a2a_seq_to_head", "ulysses_a2a_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_bwd",
     "ulysses_attn_bwd_workspace_size", "ulysses_get_device_status", "ulysses_set_wait_limit",
     "ulysses_selftest_bounded_wait", "ulysses_attn_fwd_seq", "ulysses_attn_bwd_seq", "UlyssesLayer",
-    "HostPipeline",
+    "HostPipeline", "ulysses_a2a_seq_to_head_frag", "ulysses_a2a_head_to_seq_frag",
 ]
 
 
@@ -71,6 +71,32 @@ def ulysses_a2a_head_to_seq(x0_head, x1_head, x2_head, x0_seq, x1_seq, x2_seq, N
         _ptrs(x0_head, P), _ptrs(x1_head, P), _ptrs(x2_head, P), _ptrs(x0_seq, P), _ptrs(x1_seq, P),
         _ptrs(x2_seq, P), N, P, H, H_kv, d, cu, ns, rank_lo, P if rank_hi is None else rank_hi, _stream(stream))
     check("ulysses_a2a_head_to_seq", code)
+
+
+def _one(t: Optional[torch.Tensor], dtype=torch.bfloat16):
+    if t is None:
+        return None
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"need a contiguous CUDA {dtype} tensor, got {t.dtype} on {t.device}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def ulysses_a2a_seq_to_head_frag(x0_seq, x1_seq, x2_seq, x0_frag, x1_frag, x2_frag, N, P, H, H_kv, d, head_lo,
+                                 num_heads, stream=None):
+    """Global query heads [head_lo, head_lo + num_heads) (and their kv heads)
+    of every token, from the P sequence shards into one fragment buffer each."""
+    code = lib().ulysses_a2a_seq_to_head_frag(
+        _ptrs(x0_seq, P), _ptrs(x1_seq, P), _ptrs(x2_seq, P), _one(x0_frag), _one(x1_frag), _one(x2_frag),
+        N, P, H, H_kv, d, head_lo, num_heads, _stream(stream))
+    check("ulysses_a2a_seq_to_head_frag", code)
+
+
+def ulysses_a2a_head_to_seq_frag(x0_frag, x1_frag, x2_frag, x0_seq, x1_seq, x2_seq, N, P, H, H_kv, d, head_lo,
+                                 num_heads, stream=None):
+    code = lib().ulysses_a2a_head_to_seq_frag(
+        _one(x0_frag), _one(x1_frag), _one(x2_frag), _ptrs(x0_seq, P), _ptrs(x1_seq, P), _ptrs(x2_seq, P),
+        N, P, H, H_kv, d, head_lo, num_heads, _stream(stream))
+    check("ulysses_a2a_head_to_seq_frag", code)
 
 
 def ulysses_attn_fwd(q_head, k_head, v_head, o_head, lse_head, N, P, H, H_kv, d, cu_seqlens=None,
@@ -154,7 +180,8 @@ class UlyssesLayer:
 
     def __init__(self, N: int, P: int, H: int, H_kv: int, d: int, device="cuda", cu_seqlens=None,
                  max_seqlen: int = 0, softmax_scale: float = 0.0, backward: bool = True,
-                 rank_sequential: bool = False, fused: bool = False, deterministic: bool = False):
+                 rank_sequential: bool = False, fused: bool = False, deterministic: bool = False,
+                 head_fragment: int = 0):
         if P > MAX_RANKS:
             raise ValueError(f"P <= {MAX_RANKS}")
         self.N, self.P, self.H, self.H_kv, self.d = N, P, H, H_kv, d
@@ -169,18 +196,43 @@ class UlyssesLayer:
         self.fused = fused
         if fused and (rank_sequential or (N // P) % 128 != 0):
             raise ValueError("the fused layer needs all ranks at once and N/P a multiple of 128")
+        # head_fragment = f > 0: every rank processes its heads f at a time (whole GQA
+        # groups), one fragment after another; only one fragment's full-sequence
+        # buffers exist (ulysses_a2a_*_frag + attention with P = 1 on the fragment).
+        self.frag = int(head_fragment)
+        g = H // H_kv
+        if self.frag:
+            if fused or rank_sequential:
+                raise ValueError("head_fragment excludes fused and rank_sequential")
+            if self.frag % g != 0 or (H // P) % self.frag != 0:
+                raise ValueError(f"head_fragment must be a multiple of H/H_kv = {g} dividing H/P = {H // P}")
         bf, f32 = torch.bfloat16, torch.float32
         nb = 1 if rank_sequential else P      # rank-sequential: one rank's head buffers, reused
-        if fused:
+        if fused or self.frag:
             nb = 0
         mk = lambda hx: [torch.empty(N, hx // P, d, dtype=bf, device=device) for _ in range(nb)]
         self.q_h, self.k_h, self.v_h, self.o_h = mk(H), mk(H_kv), mk(H_kv), mk(H)
-        self.lse = [torch.empty(H // P, N, dtype=f32, device=device) for _ in range(P if fused else nb)]
+        self.lse = [torch.empty(H // P, N, dtype=f32, device=device) for _ in range(P if (fused or self.frag) else nb)]
         self.backward_enabled = backward and not rank_sequential
-        if self.backward_enabled:
+        if self.frag:
+            f, fk = self.frag, self.frag // g
+            fb = lambda hx: torch.empty(N, hx, d, dtype=bf, device=device)
+            self.q_f, self.k_f, self.v_f, self.o_f = fb(f), fb(fk), fb(fk), fb(f)
+            if self.backward_enabled:
+                self.do_f, self.dq_f, self.dk_f, self.dv_f = fb(f), fb(f), fb(fk), fb(fk)
+                ws = ulysses_attn_bwd_workspace_size(N, 1, f, fk, d, deterministic)
+                self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
+        elif self.backward_enabled:
             self.do_h, self.dq_h, self.dk_h, self.dv_h = mk(H), mk(H), mk(H_kv), mk(H_kv)
             ws = ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, deterministic)
             self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
+
+    def _fragments(self):
+        """(rank, head offset within the rank, global first query head) of every fragment."""
+        hl = self.H // self.P
+        for r in range(self.P):
+            for j0 in range(0, hl, self.frag):
+                yield r, j0, r * hl + j0
 
     def _rank_bufs(self, bufs, r):
         lst = [None] * self.P
@@ -195,6 +247,15 @@ class UlyssesLayer:
             self._seq_in = (q_seq, k_seq, v_seq, o_seq)
             ulysses_attn_fwd_seq(q_seq, k_seq, v_seq, o_seq, self.lse, N, P, H, H_kv, d, self.cu, self.max_seqlen,
                                  self.scale)
+        elif self.frag:
+            self._seq_in = (q_seq, k_seq, v_seq, o_seq)
+            f, fk = self.frag, self.frag // (H // H_kv)
+            for r, j0, h_lo in self._fragments():
+                ulysses_a2a_seq_to_head_frag(q_seq, k_seq, v_seq, self.q_f, self.k_f, self.v_f, N, P, H, H_kv, d,
+                                             h_lo, f)
+                ulysses_attn_fwd([self.q_f], [self.k_f], [self.v_f], [self.o_f], [self.lse[r][j0:j0 + f]], N, 1, f,
+                                 fk, d, self.cu, self.max_seqlen, self.scale)
+                ulysses_a2a_head_to_seq_frag(self.o_f, None, None, o_seq, None, None, N, P, H, H_kv, d, h_lo, f)
         elif not self.rank_sequential:
             ulysses_a2a_seq_to_head(q_seq, k_seq, v_seq, self.q_h, self.k_h, self.v_h, N, P, H, H_kv, d, self.cu)
             ulysses_attn_fwd(self.q_h, self.k_h, self.v_h, self.o_h, self.lse, N, P, H, H_kv, d, self.cu,
@@ -219,6 +280,20 @@ class UlyssesLayer:
             dq_seq = [torch.empty(N // P, H, d, dtype=torch.bfloat16, device=do_seq[0].device) for _ in range(P)]
             dk_seq = [torch.empty(N // P, H_kv, d, dtype=torch.bfloat16, device=do_seq[0].device) for _ in range(P)]
             dv_seq = [torch.empty(N // P, H_kv, d, dtype=torch.bfloat16, device=do_seq[0].device) for _ in range(P)]
+        if self.frag:
+            q_seq, k_seq, v_seq, o_seq = self._seq_in
+            f, fk = self.frag, self.frag // (H // H_kv)
+            for r, j0, h_lo in self._fragments():
+                ulysses_a2a_seq_to_head_frag(q_seq, k_seq, v_seq, self.q_f, self.k_f, self.v_f, N, P, H, H_kv, d,
+                                             h_lo, f)
+                ulysses_a2a_seq_to_head_frag(o_seq, None, None, self.o_f, None, None, N, P, H, H_kv, d, h_lo, f)
+                ulysses_a2a_seq_to_head_frag(do_seq, None, None, self.do_f, None, None, N, P, H, H_kv, d, h_lo, f)
+                ulysses_attn_bwd([self.q_f], [self.k_f], [self.v_f], [self.o_f], [self.lse[r][j0:j0 + f]],
+                                 [self.do_f], [self.dq_f], [self.dk_f], [self.dv_f], N, 1, f, fk, d, self.workspace,
+                                 self.cu, self.max_seqlen, self.scale, deterministic=self.deterministic)
+                ulysses_a2a_head_to_seq_frag(self.dq_f, self.dk_f, self.dv_f, dq_seq, dk_seq, dv_seq, N, P, H, H_kv,
+                                             d, h_lo, f)
+            return dq_seq, dk_seq, dv_seq
         if self.fused:
             q_seq, k_seq, v_seq, o_seq = self._seq_in
             ulysses_attn_bwd_seq(q_seq, k_seq, v_seq, o_seq, self.lse, do_seq, dq_seq, dk_seq, dv_seq, N, P, H,

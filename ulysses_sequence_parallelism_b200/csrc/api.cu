@@ -81,6 +81,47 @@ uly_status a2a(bool seq_to_head, const void* const* s0, const void* const* s1, c
   return from_cuda(uly::launch_permute(seq_to_head, src, dst, hx, N, P, d, rank_lo, rank_hi, stream));
 }
 
+// A head fragment: whole GQA groups inside one rank's query heads.
+uly_status check_fragment(int64_t N, int P, int H, int H_kv, int d, int head_lo, int num_heads) {
+  uly_status st = check_shape(N, P, H, H_kv, d, 0, P);
+  if (st != ULY_OK) return st;
+  const int group = H / H_kv, hl = H / P;
+  if (num_heads < 1 || head_lo < 0 || head_lo + num_heads > H) return ULY_ERR_INVALID_ARG;
+  if (head_lo % group != 0 || num_heads % group != 0) return ULY_ERR_INVALID_ARG;
+  if (head_lo / hl != (head_lo + num_heads - 1) / hl) return ULY_ERR_INVALID_ARG;   // inside one rank
+  return ULY_OK;
+}
+
+uly_status a2a_fragment(bool seq_to_head, const void* const* seq0, const void* const* seq1,
+                        const void* const* seq2, const void* f0, const void* f1, const void* f2, int64_t N, int P,
+                        int H, int H_kv, int d, int head_lo, int num_heads, cudaStream_t stream) {
+  uly_status st = check_fragment(N, P, H, H_kv, d, head_lo, num_heads);
+  if (st != ULY_OK) return st;
+  if (seq0 == nullptr || f0 == nullptr) return ULY_ERR_INVALID_ARG;
+  if ((seq1 == nullptr) != (f1 == nullptr) || (seq2 == nullptr) != (f2 == nullptr)) return ULY_ERR_INVALID_ARG;
+  if (H * (d / 8) > uly::permute_max_row_vecs()) return ULY_ERR_UNSUPPORTED;
+  const void* const* seq[3] = {seq0, seq1, seq2};
+  const void* frag[3] = {f0, f1, f2};
+  const void* fptr[3][1] = {{f0}, {f1}, {f2}};
+  for (int s = 0; s < 3; ++s) {
+    if (seq[s] == nullptr) continue;
+    if (!ranks_ok(seq[s], 0, P) || !aligned16(frag[s])) return ULY_ERR_INVALID_ARG;
+  }
+  const int group = H / H_kv;
+  const int hx[3] = {H, H_kv, H_kv};
+  const int f_lo[3] = {head_lo, head_lo / group, head_lo / group};
+  const int f_cnt[3] = {num_heads, num_heads / group, num_heads / group};
+  const void* const* head[3] = {fptr[0], fptr[1], fptr[2]};
+  const void* const* src[3];
+  void* const* dst[3];
+  for (int s = 0; s < 3; ++s) {
+    const bool on = seq[s] != nullptr;
+    src[s] = !on ? nullptr : (seq_to_head ? seq[s] : head[s]);
+    dst[s] = !on ? nullptr : const_cast<void* const*>(seq_to_head ? head[s] : seq[s]);
+  }
+  return from_cuda(uly::launch_permute_fragment(seq_to_head, src, dst, hx, f_lo, f_cnt, N, P, d, stream));
+}
+
 float resolve_scale(float softmax_scale, int d) {
   return (softmax_scale > 0.f && isfinite(softmax_scale)) ? softmax_scale : 1.0f / sqrtf(static_cast<float>(d));
 }
@@ -104,6 +145,23 @@ uly_status ulysses_a2a_head_to_seq(const void* const* x0_head, const void* const
                                    cudaStream_t stream) {
   return a2a(false, x0_head, x1_head, x2_head, x0_seq, x1_seq, x2_seq, N, P, H, H_kv, d, cu_seqlens, num_seqs,
              rank_lo, rank_hi, stream);
+}
+
+uly_status ulysses_a2a_seq_to_head_frag(const void* const* x0_seq, const void* const* x1_seq,
+                                        const void* const* x2_seq, void* x0_frag, void* x1_frag, void* x2_frag,
+                                        int64_t N, int P, int H, int H_kv, int d, int head_lo, int num_heads,
+                                        cudaStream_t stream) {
+  return a2a_fragment(true, x0_seq, x1_seq, x2_seq, x0_frag, x1_frag, x2_frag, N, P, H, H_kv, d, head_lo, num_heads,
+                      stream);
+}
+
+uly_status ulysses_a2a_head_to_seq_frag(const void* x0_frag, const void* x1_frag, const void* x2_frag,
+                                        void* const* x0_seq, void* const* x1_seq, void* const* x2_seq, int64_t N,
+                                        int P, int H, int H_kv, int d, int head_lo, int num_heads,
+                                        cudaStream_t stream) {
+  auto cv = [](void* const* p) { return reinterpret_cast<const void* const*>(p); };
+  return a2a_fragment(false, cv(x0_seq), cv(x1_seq), cv(x2_seq), x0_frag, x1_frag, x2_frag, N, P, H, H_kv, d,
+                      head_lo, num_heads, stream);
 }
 
 uly_status ulysses_attn_fwd(const void* const* q_head, const void* const* k_head, const void* const* v_head,

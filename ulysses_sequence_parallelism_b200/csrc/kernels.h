@@ -20,6 +20,12 @@ struct AttnShape {
 int permute_max_row_vecs();
 cudaError_t launch_permute(bool seq_to_head, const void* const* src[3], void* const* dst[3], const int hx[3],
                            int64_t N, int P, int d, int rank_lo, int rank_hi, cudaStream_t stream);
+// One head fragment per slot: global heads [f_lo[s], f_lo[s] + f_cnt[s]) of
+// tensor s between the P sequence shards and the single head-side buffer at
+// index 0 of the head-side pointer array ([N, f_cnt[s], d]).
+cudaError_t launch_permute_fragment(bool seq_to_head, const void* const* src[3], void* const* dst[3],
+                                    const int hx[3], const int f_lo[3], const int f_cnt[3], int64_t N, int P, int d,
+                                    cudaStream_t stream);
 
 cudaError_t launch_attn_fwd(const AttnShape& s, const void* const* q, const void* const* k,
                             const void* const* v, void* const* o, float* const* lse, cudaStream_t stream);

@@ -6,6 +6,10 @@
 // become, with the P ranks as P buffers of one GPU, pure index maps:
 //   seq -> head : head[q][t, j, :] = seq[t / n][t % n, q*Hl + j, :]   (n = N/P, Hl = Hx/P)
 //   head -> seq : the inverse.
+// The same kernel moves a head fragment of one rank (a whole number of GQA
+// groups, processed one after another to shrink activation memory:
+// q2bstudio.com, "Ulysses Unleashed", fragmentation by heads): then the head
+// side is one buffer [N, f, d] holding global heads [h_lo, h_lo + f).
 // HBM-bound: every byte is read once and written once. The kernel walks the
 // sequence-side rows (one token of one rank: Hx*d contiguous bf16), so the
 // sequence side is streamed contiguously and the head side is written/read in
@@ -28,7 +32,10 @@ constexpr int kTargetBlocks = 148 * 8;  // ~2 waves of 4 resident 512-thread blo
 struct SlotArgs {
   RankPtrs src;
   RankPtrsMut dst;
-  int hx;          // heads of this tensor (H or H_kv)
+  int hx;          // heads of this tensor on the sequence side (H or H_kv)
+  int hb;          // heads per head-side buffer (Hx/P, or the fragment size)
+  int h_lo, h_cnt; // global heads moved: [h_lo, h_lo + h_cnt)
+  int h_base;      // head-side buffer b holds global heads [h_base + b*hb, +hb)
   int active;
 };
 
@@ -38,7 +45,6 @@ struct PermuteArgs {
   int n;           // tokens per rank (N/P)
   int P;
   int dvec;        // d / 8 : 16-byte vectors per head row
-  int rank_lo, rank_hi;
   int rows_per_block;
 };
 
@@ -58,11 +64,11 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(const __grid_constant
   const int yi = blockIdx.y / a.P;
   const int p = blockIdx.y - yi * a.P;               // sequence-side rank
   const SlotArgs& sl = a.slot[a.slot_of[yi]];
-  const int Hl = sl.hx / a.P;
+  const int Hl = sl.hb;
   const int row_vecs = sl.hx * a.dvec;                // vectors per sequence-side row
   const int head_row_vecs = Hl * a.dvec;              // vectors per head-side token row
-  const int lo_v = a.rank_lo * head_row_vecs;
-  const int rv = (a.rank_hi - a.rank_lo) * head_row_vecs;
+  const int lo_v = sl.h_lo * a.dvec;
+  const int rv = sl.h_cnt * a.dvec;
 
   // Column assignment: rows_per_pass rows per pass, vpt vectors per thread per row.
   int rows_per_pass, vpt, r_off;
@@ -87,8 +93,8 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(const __grid_constant
     int vv = lo_v + v;
     int hx = vv / a.dvec;
     int c = vv - hx * a.dvec;
-    int q = hx / Hl;
-    int j = hx - q * Hl;
+    int q = (hx - sl.h_base) / Hl;
+    int j = hx - sl.h_base - q * Hl;
     seq_off[k] = ok ? vv : -1;
     q_of[k] = q;
     head_off[k] = j * a.dvec + c;
@@ -146,32 +152,40 @@ __global__ void __launch_bounds__(kThreads) permute_kernel(const __grid_constant
 int permute_max_row_vecs() {
   using namespace permute_impl; return kThreads * kMaxVecPerThread; }
 
-cudaError_t launch_permute(bool seq_to_head, const void* const* src[3], void* const* dst[3], const int hx[3],
-                           int64_t N, int P, int d, int rank_lo, int rank_hi, cudaStream_t stream) {
-  using namespace permute_impl;
+namespace permute_impl {
+// hb/h_lo/h_cnt/h_base per slot as in SlotArgs; nb = head-side buffers used
+// (indices [b_lo, b_lo + nb) of the head-side pointer arrays).
+cudaError_t launch(bool seq_to_head, const void* const* src[3], void* const* dst[3], const int hx[3],
+                   const int hb[3], const int h_lo[3], const int h_cnt[3], const int h_base[3], int b_lo, int nb,
+                   int64_t N, int P, int d, cudaStream_t stream) {
   PermuteArgs a;
   memset(&a, 0, sizeof(a));
   a.n = static_cast<int>(N / P);
   a.P = P;
   a.dvec = d / 8;
-  a.rank_lo = rank_lo;
-  a.rank_hi = rank_hi;
   int max_rows_per_pass = 1;
   int n_active = 0;
   for (int s = 0; s < 3; ++s) {
-    a.slot[s].active = (src[s] != nullptr && dst[s] != nullptr) ? 1 : 0;
-    a.slot[s].hx = hx[s];
-    if (!a.slot[s].active) continue;
+    SlotArgs& sl = a.slot[s];
+    sl.active = (src[s] != nullptr && dst[s] != nullptr) ? 1 : 0;
+    sl.hx = hx[s];
+    sl.hb = hb[s];
+    sl.h_lo = h_lo[s];
+    sl.h_cnt = h_cnt[s];
+    sl.h_base = h_base[s];
+    if (!sl.active) continue;
     a.slot_of[n_active++] = s;
-    const bool sr = seq_to_head;
+    const void* const* seq_side = seq_to_head ? src[s] : dst[s];
+    const void* const* head_side = seq_to_head ? dst[s] : src[s];
     for (int r = 0; r < P; ++r) {
-      // sequence-side buffers: every rank; head-side buffers: ranks in range only.
-      bool need_src = sr ? true : (r >= rank_lo && r < rank_hi);
-      bool need_dst = sr ? (r >= rank_lo && r < rank_hi) : true;
-      a.slot[s].src.p[r] = need_src ? src[s][r] : nullptr;
-      a.slot[s].dst.p[r] = need_dst ? dst[s][r] : nullptr;
+      if (seq_to_head) sl.src.p[r] = seq_side[r];
+      else sl.dst.p[r] = const_cast<void*>(seq_side[r]);
     }
-    int rv = (rank_hi - rank_lo) * (hx[s] / P) * (d / 8);
+    for (int b = b_lo; b < b_lo + nb; ++b) {      // head-side buffers in use only
+      if (seq_to_head) sl.dst.p[b] = const_cast<void*>(head_side[b]);
+      else sl.src.p[b] = head_side[b];
+    }
+    int rv = h_cnt[s] * (d / 8);
     int rpp = rv <= kThreads ? kThreads / rv : 1;
     if (rpp > max_rows_per_pass) max_rows_per_pass = rpp;
   }
@@ -188,6 +202,27 @@ cudaError_t launch_permute(bool seq_to_head, const void* const* src[3], void* co
   else
     permute_kernel<false><<<grid, kThreads, 0, stream>>>(a);
   return cudaGetLastError();
+}
+}  // namespace permute_impl
+
+cudaError_t launch_permute(bool seq_to_head, const void* const* src[3], void* const* dst[3], const int hx[3],
+                           int64_t N, int P, int d, int rank_lo, int rank_hi, cudaStream_t stream) {
+  int hb[3], h_lo[3], h_cnt[3], h_base[3] = {0, 0, 0};
+  for (int s = 0; s < 3; ++s) {
+    hb[s] = hx[s] / P;
+    h_lo[s] = rank_lo * hb[s];
+    h_cnt[s] = (rank_hi - rank_lo) * hb[s];
+  }
+  return permute_impl::launch(seq_to_head, src, dst, hx, hb, h_lo, h_cnt, h_base, rank_lo, rank_hi - rank_lo, N, P,
+                              d, stream);
+}
+
+cudaError_t launch_permute_fragment(bool seq_to_head, const void* const* src[3], void* const* dst[3],
+                                    const int hx[3], const int f_lo[3], const int f_cnt[3], int64_t N, int P, int d,
+                                    cudaStream_t stream) {
+  int h_base[3];
+  for (int s = 0; s < 3; ++s) h_base[s] = f_lo[s];
+  return permute_impl::launch(seq_to_head, src, dst, hx, f_cnt, f_lo, f_cnt, h_base, 0, 1, N, P, d, stream);
 }
 
 }  // namespace uly
