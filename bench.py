@@ -445,6 +445,44 @@ def main():
                 "head_side_bytes_unfragmented": full_bytes}
         del lfr
 
+    # ---------------------------------------------------------------- projections (NEXT-4)
+    # QKV projection storing straight into the head shards and output projection
+    # reading straight from them (hidden = H d, synthetic seeded weights)
+    proj = None
+    if not w.rank_sequential and (N // P) % 128 == 0:
+        hidden = H * d
+        xb, wqb, wob = workloads.projection_inputs(N, H, H_kv, d, hidden, seed=1)
+        tdev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        x_seq = [tdev(a) for a in workloads.seq_shards(xb, P)]
+        w_qkv, w_o = tdev(wqb), tdev(wob)
+        y_seq = [torch.empty_like(t) for t in x_seq]
+        del xb, wqb, wob
+        L = layer
+
+        def timed(fn, reps=5):
+            for _ in range(2):
+                fn()
+            ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ea.record(stream)
+            for _ in range(reps):
+                fn()
+            eb.record(stream)
+            torch.cuda.synchronize()
+            return ea.elapsed_time(eb) / reps
+
+        qkv_ms = timed(lambda: U.ulysses_qkv_proj_seq_to_head(x_seq, w_qkv, L.q_h, L.k_h, L.v_h, N, P, H, H_kv, d,
+                                                               hidden))
+        out_ms = timed(lambda: U.ulysses_out_proj_head_to_seq(L.o_h, w_o, y_seq, N, P, H, H_kv, d, hidden))
+        blk_ms = timed(lambda: L.forward_projected(x_seq, w_qkv, w_o, y_seq), reps=3)
+        f_qkv = 2.0 * N * hidden * (H + 2 * H_kv) * d
+        f_out = 2.0 * N * H * d * hidden
+        proj = {"hidden": hidden, "qkv_proj_ms": qkv_ms, "qkv_proj_tflops": f_qkv / (qkv_ms / 1e3) / 1e12,
+                "out_proj_ms": out_ms, "out_proj_tflops": f_out / (out_ms / 1e3) / 1e12,
+                "block_fwd_ms": blk_ms, "block_fwd_tokens_per_s": N / (blk_ms / 1e3),
+                "note": "forward block = QKV projection into head shards + attention + output projection "
+                        "from head shards (no permute launches)"}
+        del x_seq, y_seq, w_qkv, w_o
+
     # ---------------------------------------------------------------- end to end through the public API
     # HostPipeline: every step copies its inputs from pinned host memory and
     # reads its results back; copies of neighbouring steps overlap the kernels.
@@ -501,7 +539,7 @@ def main():
                        "parallelism": f"{P} virtual ranks per GPU; {world} independent replica(s)"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk, "detail": detail, "fused": fused, "head_fragment": frag,
+            "clocks": clk, "detail": detail, "fused": fused, "head_fragment": frag, "projections": proj,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -122,6 +122,32 @@ ULY_API uly_status ulysses_a2a_head_to_seq_frag(
     void* const* x0_seq, void* const* x1_seq, void* const* x2_seq,
     int64_t N, int P, int H, int H_kv, int d, int head_lo, int num_heads, cudaStream_t stream);
 
+/* The projections on either side of the exchange, with the all-to-alls folded
+ * into the GEMMs (each rank projects its own tokens before the first
+ * all-to-all and its own shard after the second: theaicatchup.com, "How Does
+ * Ulysses Sequence Parallelism Actually Work?").
+ * ulysses_qkv_proj_seq_to_head: for every token t of every sequence shard,
+ *   [q_t | k_t | v_t] = x_t W_qkv^T  (fp32 accumulation, bf16 round to nearest
+ *   even), with x_seq[p] [N/P, hidden], w_qkv [(H + 2 H_kv) d, hidden]
+ *   row-major (rows 0..H d-1 give Q heads in order, then K heads, then V
+ *   heads), written straight into the head shards q_head/k_head/v_head of all
+ *   P ranks ([N, H/P, d] and [N, H_kv/P, d]): the same result as projecting
+ *   into sequence shards and calling ulysses_a2a_seq_to_head.
+ * ulysses_out_proj_head_to_seq: y_t = o_t W_o^T with o_t gathered from the
+ *   head shards o_head (all P ranks) and w_o [hidden, H d], written into the
+ *   sequence shards y_seq[p] [N/P, hidden]: the same result as
+ *   ulysses_a2a_head_to_seq followed by the projection.
+ * Needs (N/P) % 128 == 0, hidden % 256 == 0 and (H + 2 H_kv) d % 256 == 0
+ * (else ULY_ERR_UNSUPPORTED); other shape rules as the layer. All pointers
+ * 16-byte aligned device memory owned by the caller; asynchronous. */
+ULY_API uly_status ulysses_qkv_proj_seq_to_head(
+    const void* const* x_seq, const void* w_qkv,
+    void* const* q_head, void* const* k_head, void* const* v_head,
+    int64_t N, int P, int H, int H_kv, int d, int hidden, cudaStream_t stream);
+ULY_API uly_status ulysses_out_proj_head_to_seq(
+    const void* const* o_head, const void* w_o, void* const* y_seq,
+    int64_t N, int P, int H, int H_kv, int d, int hidden, cudaStream_t stream);
+
 /* Causal (optionally packed-varlen) grouped-query flash attention forward on the
  * head shards of ranks [rank_lo, rank_hi): each rank runs attention by itself on
  * its heads, which do not interact (theaicatchup.com, ibid., citing DeepSpeed-Ulysses):

@@ -16,6 +16,7 @@ Modules:
                 sampled-column variants for the large workloads
   layer      -- the Ulysses layer as the pages' steps: a2a, attention, a2a
   brute      -- pure-Python triple-loop attention for tiny inputs (a pin)
+  projection -- the QKV and output projections either side of the exchange
 
 Every function pinned by tests in ``tests/test_oracle_pins.py``; there is no
 unpinned function.
@@ -25,8 +26,9 @@ from .permute import seq_to_head, head_to_seq
 from .attention import (doc_starts, doc_ends, attention_forward, attention_backward,
                         bwd_preprocess, attention_rows, attention_kv_cols)
 from .layer import ulysses_layer_forward, ulysses_layer_backward
+from .projection import qkv_projection, out_projection
 
 __all__ = ["widen_bf16", "seq_to_head", "head_to_seq", "doc_starts", "doc_ends",
            "attention_forward", "attention_backward", "bwd_preprocess",
            "attention_rows", "attention_kv_cols",
-           "ulysses_layer_forward", "ulysses_layer_backward"]
+           "ulysses_layer_forward", "ulysses_layer_backward", "qkv_projection", "out_projection"]

@@ -150,3 +150,20 @@ def test_fragment_entry_points_validate_before_launch(L):
                                           None) == 1
     # unsupported head dim
     assert L.ulysses_a2a_seq_to_head_frag(p, None, None, f, None, None, N, P, H, H_kv, 96, 0, 4, None) == 2
+
+
+def test_projection_entry_points_validate_before_launch(L):
+    P = 2
+    p = _arr([GOOD] * P)
+    w = ctypes.c_void_p(GOOD)
+    # hidden not a multiple of 256, rows per shard not a multiple of 128: unsupported
+    assert L.ulysses_qkv_proj_seq_to_head(p, w, p, p, p, 512, P, 8, 2, 128, 1000, None) == 2
+    assert L.ulysses_qkv_proj_seq_to_head(p, w, p, p, p, 400, P, 8, 2, 128, 1024, None) == 2
+    assert L.ulysses_out_proj_head_to_seq(p, w, p, 400, P, 8, 2, 128, 1024, None) == 2
+    # (H + 2 H_kv) d not a multiple of 256
+    assert L.ulysses_qkv_proj_seq_to_head(p, w, p, p, p, 512, P, 2, 2, 64, 1024, None) == 2
+    # misaligned weight, missing shard pointer, bad hidden
+    assert L.ulysses_qkv_proj_seq_to_head(p, ctypes.c_void_p(GOOD + 2), p, p, p, 512, P, 8, 2, 128, 1024,
+                                          None) == 1
+    assert L.ulysses_out_proj_head_to_seq(_arr([GOOD, 0]), w, p, 512, P, 8, 2, 128, 1024, None) == 1
+    assert L.ulysses_out_proj_head_to_seq(p, w, p, 512, P, 8, 2, 128, 0, None) == 1

@@ -341,3 +341,82 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(oatt, "doc_starts", orig_starts)
     monkeypatch.setattr(oatt, "_scale", lambda d_, s: 1.0)                               # wrong scale
     assert differs()
+
+
+# ---------------------------------------------------------------- projections (NEXT-4)
+
+def _brute_matvec(x_row, w):
+    """Pure-Python y_j = fsum_c x_c w[j][c]."""
+    import math
+    return [math.fsum(float(a) * float(b) for a, b in zip(x_row, w_row)) for w_row in w]
+
+
+def test_qkv_projection_matches_brute_force_and_splits_heads_in_order():
+    import oracle
+    rng = np.random.Generator(np.random.PCG64(71))
+    P, n, hidden, H, H_kv, d = 2, 3, 5, 4, 2, 2
+    x_seq = [rng.standard_normal((n, hidden)) for _ in range(P)]
+    w = rng.standard_normal(((H + 2 * H_kv) * d, hidden))
+    q, k, v = oracle.qkv_projection(x_seq, w, H, H_kv, d)
+    for p in range(P):
+        for s in range(n):
+            y = _brute_matvec(x_seq[p][s], w)
+            for h in range(H):
+                assert np.allclose(q[p][s, h], y[h * d:(h + 1) * d], rtol=0, atol=1e-12)
+            for h in range(H_kv):
+                assert np.allclose(k[p][s, h], y[(H + h) * d:(H + h + 1) * d], rtol=0, atol=1e-12)
+                assert np.allclose(v[p][s, h], y[(H + H_kv + h) * d:(H + H_kv + h + 1) * d], rtol=0, atol=1e-12)
+
+
+def test_qkv_projection_selection_weights_route_inputs():
+    """W_qkv made of unit rows picks input features: Q head h dim c must be
+    x[(h*d + c) % hidden], K and V shifted by 1 and 2: pins row order and the
+    head/dim reshape (a transposed or mis-split W fails)."""
+    import oracle
+    P, n, H, H_kv, d = 2, 4, 4, 2, 3
+    hidden = 7
+    rng = np.random.Generator(np.random.PCG64(72))
+    x_seq = [rng.standard_normal((n, hidden)) for _ in range(P)]
+    rows = (H + 2 * H_kv) * d
+    w = np.zeros((rows, hidden))
+    src = []
+    for r in range(rows):
+        shift = 0 if r < H * d else (1 if r < (H + H_kv) * d else 2)
+        c = (r + shift) % hidden
+        w[r, c] = 1.0
+        src.append(c)
+    q, k, v = oracle.qkv_projection(x_seq, w, H, H_kv, d)
+    for p in range(P):
+        for h in range(H):
+            for c in range(d):
+                assert np.array_equal(q[p][:, h, c], x_seq[p][:, src[h * d + c]])
+        for h in range(H_kv):
+            for c in range(d):
+                assert np.array_equal(k[p][:, h, c], x_seq[p][:, src[(H + h) * d + c]])
+                assert np.array_equal(v[p][:, h, c], x_seq[p][:, src[(H + H_kv + h) * d + c]])
+
+
+def test_out_projection_identity_and_brute_force():
+    import oracle
+    rng = np.random.Generator(np.random.PCG64(73))
+    P, n, H, d = 2, 3, 2, 3
+    o_seq = [rng.standard_normal((n, H, d)) for _ in range(P)]
+    y = oracle.out_projection(o_seq, np.eye(H * d))
+    for p in range(P):
+        assert np.array_equal(y[p], o_seq[p].reshape(n, H * d))        # identity: heads concatenated in order
+    w = rng.standard_normal((5, H * d))
+    y = oracle.out_projection(o_seq, w)
+    for p in range(P):
+        for s in range(n):
+            assert np.allclose(y[p][s], _brute_matvec(o_seq[p][s].reshape(-1), w), rtol=0, atol=1e-12)
+
+
+def test_projection_planted_transpose_is_caught():
+    """A plausible mistake (x @ w instead of x @ w.T, on a square W) must fail
+    the brute-force pin above."""
+    rng = np.random.Generator(np.random.PCG64(74))
+    x = rng.standard_normal((3, 4))
+    w = rng.standard_normal((4, 4))
+    wrong = x @ w
+    right = np.array([_brute_matvec(r, w) for r in x])
+    assert not np.allclose(wrong, right, atol=1e-6)

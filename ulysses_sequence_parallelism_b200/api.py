@@ -22,6 +22,7 @@ __all__ = [
     "ulysses_attn_bwd_workspace_size", "ulysses_get_device_status", "ulysses_set_wait_limit",
     "ulysses_selftest_bounded_wait", "ulysses_attn_fwd_seq", "ulysses_attn_bwd_seq", "UlyssesLayer",
     "HostPipeline", "ulysses_a2a_seq_to_head_frag", "ulysses_a2a_head_to_seq_frag",
+    "ulysses_qkv_proj_seq_to_head", "ulysses_out_proj_head_to_seq",
 ]
 
 
@@ -97,6 +98,21 @@ def ulysses_a2a_head_to_seq_frag(x0_frag, x1_frag, x2_frag, x0_seq, x1_seq, x2_s
         _one(x0_frag), _one(x1_frag), _one(x2_frag), _ptrs(x0_seq, P), _ptrs(x1_seq, P), _ptrs(x2_seq, P),
         N, P, H, H_kv, d, head_lo, num_heads, _stream(stream))
     check("ulysses_a2a_head_to_seq_frag", code)
+
+
+def ulysses_qkv_proj_seq_to_head(x_seq, w_qkv, q_head, k_head, v_head, N, P, H, H_kv, d, hidden, stream=None):
+    """[Q|K|V] = X W_qkv^T for every token, stored straight into the head shards."""
+    code = lib().ulysses_qkv_proj_seq_to_head(
+        _ptrs(x_seq, P), _one(w_qkv), _ptrs(q_head, P), _ptrs(k_head, P), _ptrs(v_head, P), N, P, H, H_kv, d,
+        hidden, _stream(stream))
+    check("ulysses_qkv_proj_seq_to_head", code)
+
+
+def ulysses_out_proj_head_to_seq(o_head, w_o, y_seq, N, P, H, H_kv, d, hidden, stream=None):
+    """Y = O W_o^T for every token, O read straight from the head shards."""
+    code = lib().ulysses_out_proj_head_to_seq(
+        _ptrs(o_head, P), _one(w_o), _ptrs(y_seq, P), N, P, H, H_kv, d, hidden, _stream(stream))
+    check("ulysses_out_proj_head_to_seq", code)
 
 
 def ulysses_attn_fwd(q_head, k_head, v_head, o_head, lse_head, N, P, H, H_kv, d, cu_seqlens=None,
@@ -226,6 +242,24 @@ class UlyssesLayer:
             self.do_h, self.dq_h, self.dk_h, self.dv_h = mk(H), mk(H), mk(H_kv), mk(H_kv)
             ws = ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, deterministic)
             self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
+
+    def forward_projected(self, x_seq: List[torch.Tensor], w_qkv: torch.Tensor, w_o: torch.Tensor,
+                          y_seq: Optional[List[torch.Tensor]] = None):
+        """The attention block forward with its projections: hidden states
+        x_seq[p] [N/P, hidden] -> y_seq[p] [N/P, hidden]. The QKV projection
+        stores Q/K/V straight into the head shards and the output projection
+        reads O straight from them, so neither all-to-all runs as a permute."""
+        if self.fused or self.frag or self.rank_sequential:
+            raise ValueError("forward_projected runs on the plain all-ranks layer")
+        N, P, H, H_kv, d = self.N, self.P, self.H, self.H_kv, self.d
+        hidden = x_seq[0].shape[1]
+        if y_seq is None:
+            y_seq = [torch.empty_like(x) for x in x_seq]
+        ulysses_qkv_proj_seq_to_head(x_seq, w_qkv, self.q_h, self.k_h, self.v_h, N, P, H, H_kv, d, hidden)
+        ulysses_attn_fwd(self.q_h, self.k_h, self.v_h, self.o_h, self.lse, N, P, H, H_kv, d, self.cu,
+                         self.max_seqlen, self.scale)
+        ulysses_out_proj_head_to_seq(self.o_h, w_o, y_seq, N, P, H, H_kv, d, hidden)
+        return y_seq
 
     def _fragments(self):
         """(rank, head offset within the rank, global first query head) of every fragment."""

@@ -122,6 +122,15 @@ uly_status a2a_fragment(bool seq_to_head, const void* const* seq0, const void* c
   return from_cuda(uly::launch_permute_fragment(seq_to_head, src, dst, hx, f_lo, f_cnt, N, P, d, stream));
 }
 
+uly_status check_proj(int64_t N, int P, int H, int H_kv, int d, int hidden) {
+  uly_status st = check_shape(N, P, H, H_kv, d, 0, P);
+  if (st != ULY_OK) return st;
+  if (hidden <= 0) return ULY_ERR_INVALID_ARG;
+  if ((N / P) % 128 != 0 || hidden % 256 != 0 || ((H + 2 * H_kv) * d) % 256 != 0) return ULY_ERR_UNSUPPORTED;
+  if ((N / P) * static_cast<int64_t>(hidden) >= (int64_t(1) << 31)) return ULY_ERR_UNSUPPORTED;
+  return ULY_OK;
+}
+
 float resolve_scale(float softmax_scale, int d) {
   return (softmax_scale > 0.f && isfinite(softmax_scale)) ? softmax_scale : 1.0f / sqrtf(static_cast<float>(d));
 }
@@ -162,6 +171,27 @@ uly_status ulysses_a2a_head_to_seq_frag(const void* x0_frag, const void* x1_frag
   auto cv = [](void* const* p) { return reinterpret_cast<const void* const*>(p); };
   return a2a_fragment(false, cv(x0_seq), cv(x1_seq), cv(x2_seq), x0_frag, x1_frag, x2_frag, N, P, H, H_kv, d,
                       head_lo, num_heads, stream);
+}
+
+uly_status ulysses_qkv_proj_seq_to_head(const void* const* x_seq, const void* w_qkv, void* const* q_head,
+                                        void* const* k_head, void* const* v_head, int64_t N, int P, int H,
+                                        int H_kv, int d, int hidden, cudaStream_t stream) {
+  uly_status st = check_proj(N, P, H, H_kv, d, hidden);
+  if (st != ULY_OK) return st;
+  auto cv = [](void* const* p) { return reinterpret_cast<const void* const*>(p); };
+  if (!ranks_ok(x_seq, 0, P) || !aligned16(w_qkv) || !ranks_ok(cv(q_head), 0, P) || !ranks_ok(cv(k_head), 0, P) ||
+      !ranks_ok(cv(v_head), 0, P))
+    return ULY_ERR_INVALID_ARG;
+  return from_cuda(uly::launch_proj(0, x_seq, w_qkv, q_head, k_head, v_head, N, P, H, H_kv, d, hidden, stream));
+}
+
+uly_status ulysses_out_proj_head_to_seq(const void* const* o_head, const void* w_o, void* const* y_seq, int64_t N,
+                                        int P, int H, int H_kv, int d, int hidden, cudaStream_t stream) {
+  uly_status st = check_proj(N, P, H, H_kv, d, hidden);
+  if (st != ULY_OK) return st;
+  if (!ranks_ok(o_head, 0, P) || !aligned16(w_o) || !ranks_ok(reinterpret_cast<const void* const*>(y_seq), 0, P))
+    return ULY_ERR_INVALID_ARG;
+  return from_cuda(uly::launch_proj(1, o_head, w_o, y_seq, nullptr, nullptr, N, P, H, H_kv, d, hidden, stream));
 }
 
 uly_status ulysses_attn_fwd(const void* const* q_head, const void* const* k_head, const void* const* v_head,

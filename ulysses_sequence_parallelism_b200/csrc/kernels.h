@@ -47,4 +47,12 @@ cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void
                             const void* const* dO, void* const* dq, void* const* dk, void* const* dv,
                             void* workspace, int deterministic, cudaStream_t stream);
 
+// Projections with the all-to-alls folded in. mode 0: a_bufs = X sequence
+// shards [N/P, hidden], w = W_qkv [(H + 2 H_kv) d, hidden], out0/1/2 = Q/K/V
+// head shards of all P ranks. mode 1: a_bufs = O head shards [N, H/P, d],
+// w = W_o [hidden, H d], out0 = Y sequence shards [N/P, hidden].
+cudaError_t launch_proj(int mode, const void* const* a_bufs, const void* w, void* const* out0, void* const* out1,
+                        void* const* out2, int64_t N, int P, int H, int H_kv, int d, int hidden,
+                        cudaStream_t stream);
+
 }  // namespace uly

@@ -4,5 +4,6 @@
 #include "permute.cu"
 #include "attn_fwd_sm100.cu"
 #include "attn_bwd_sm100.cu"
+#include "proj_sm100.cu"
 #include "api.cu"
 #include "bwd_noalloc.cu"

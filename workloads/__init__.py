@@ -144,3 +144,15 @@ def causal_pairs(N: int, cu_seqlens=None) -> int:
         return N * (N + 1) // 2
     L = np.diff(np.asarray(cu_seqlens, dtype=np.int64))
     return int(np.sum(L * (L + 1) // 2))
+
+
+def projection_inputs(N: int, H: int, H_kv: int, d: int, hidden: int, seed: int = 1):
+    """Seeded synthetic hidden states and projection weights (bf16 bit
+    patterns): x [N, hidden] ~ N(0, 1); W_qkv [(H + 2 H_kv) d, hidden] and
+    W_o [hidden, H d] ~ N(0, 1/fan_in), so projected values stay O(1). One
+    PCG64(seed) stream in the order x, W_qkv, W_o. No arithmetic of the method."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = _draw_bf16(rng, (N, hidden), 1.0)
+    w_qkv = _draw_bf16(rng, ((H + 2 * H_kv) * d, hidden), 1.0 / math.sqrt(hidden))
+    w_o = _draw_bf16(rng, (hidden, H * d), 1.0 / math.sqrt(H * d))
+    return x, w_qkv, w_o
