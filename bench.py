@@ -479,8 +479,26 @@ def main():
         proj = {"hidden": hidden, "qkv_proj_ms": qkv_ms, "qkv_proj_tflops": f_qkv / (qkv_ms / 1e3) / 1e12,
                 "out_proj_ms": out_ms, "out_proj_tflops": f_out / (out_ms / 1e3) / 1e12,
                 "block_fwd_ms": blk_ms, "block_fwd_tokens_per_s": N / (blk_ms / 1e3),
-                "note": "forward block = QKV projection into head shards + attention + output projection "
-                        "from head shards (no permute launches)"}
+                "note": "block = QKV projection into head shards + attention + output projection from head "
+                        "shards, and the gradients of all three (no permute launches)"}
+        if w.backward:
+            dy_seq = [torch.randn_like(t, dtype=torch.float32).to(torch.bfloat16) for t in y_seq]
+            dw_o, dw_qkv = torch.empty_like(w_o), torch.empty_like(w_qkv)
+            dx_seq = [torch.empty_like(t) for t in x_seq]
+            obwd_ms = timed(lambda: U.ulysses_out_proj_bwd(L.o_h, w_o, dy_seq, L.do_h, dw_o, N, P, H, H_kv, d,
+                                                           hidden))
+            qbwd_ms = timed(lambda: U.ulysses_qkv_proj_bwd(x_seq, w_qkv, L.dq_h, L.dk_h, L.dv_h, dx_seq, dw_qkv, N,
+                                                           P, H, H_kv, d, hidden))
+
+            def block_step():
+                L.forward_projected(x_seq, w_qkv, w_o, y_seq)
+                L.backward_projected(dy_seq, x_seq, w_qkv, w_o)
+
+            full_ms = timed(block_step, reps=3)
+            proj.update({"out_proj_bwd_ms": obwd_ms, "out_proj_bwd_tflops": 2 * f_out / (obwd_ms / 1e3) / 1e12,
+                         "qkv_proj_bwd_ms": qbwd_ms, "qkv_proj_bwd_tflops": 2 * f_qkv / (qbwd_ms / 1e3) / 1e12,
+                         "block_fwd_bwd_ms": full_ms, "block_fwd_bwd_tokens_per_s": N / (full_ms / 1e3)})
+            del dy_seq, dw_o, dw_qkv, dx_seq
         del x_seq, y_seq, w_qkv, w_o
 
     # ---------------------------------------------------------------- end to end through the public API

@@ -148,6 +148,32 @@ ULY_API uly_status ulysses_out_proj_head_to_seq(
     const void* const* o_head, const void* w_o, void* const* y_seq,
     int64_t N, int P, int H, int H_kv, int d, int hidden, cudaStream_t stream);
 
+/* Backward of the two projections (the gradient of the formulas above; the
+ * pages train through the block but do not write its backward), with the
+ * all-to-alls again folded into the GEMMs' loads and stores:
+ * ulysses_out_proj_bwd: from dy_seq[p] [N/P, hidden] (gradient of Y),
+ *   do_head = dY W_o written straight into the head shards ([N, H/P, d] per
+ *   rank: the input of ulysses_attn_bwd, no seq->head permute of dO), and
+ *   dw_o = sum over all tokens of dy_t^T o_t  ([hidden, H d]), with O read
+ *   from the head shards o_head.
+ * ulysses_qkv_proj_bwd: from the attention gradients dq_head, dk_head, dv_head
+ *   (head shards, as ulysses_attn_bwd writes them), dx_seq[p] = [dq|dk|dv]_t
+ *   W_qkv (sequence shards [N/P, hidden]: no head->seq permute of dQ, dK, dV),
+ *   and dw_qkv = sum over all tokens of [dq|dk|dv]_t^T x_t
+ *   ([(H + 2 H_kv) d, hidden]).
+ * fp32 accumulation over the whole reduction, one bf16 rounding (RNE). Weight
+ * gradients are written, not accumulated into. Shape rules as the forward
+ * projections; ulysses_out_proj_bwd also needs H d % 256 == 0. */
+ULY_API uly_status ulysses_out_proj_bwd(
+    const void* const* o_head, const void* w_o, const void* const* dy_seq,
+    void* const* do_head, void* dw_o,
+    int64_t N, int P, int H, int H_kv, int d, int hidden, cudaStream_t stream);
+ULY_API uly_status ulysses_qkv_proj_bwd(
+    const void* const* x_seq, const void* w_qkv,
+    const void* const* dq_head, const void* const* dk_head, const void* const* dv_head,
+    void* const* dx_seq, void* dw_qkv,
+    int64_t N, int P, int H, int H_kv, int d, int hidden, cudaStream_t stream);
+
 /* Causal (optionally packed-varlen) grouped-query flash attention forward on the
  * head shards of ranks [rank_lo, rank_hi): each rank runs attention by itself on
  * its heads, which do not interact (theaicatchup.com, ibid., citing DeepSpeed-Ulysses):

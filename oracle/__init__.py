@@ -26,9 +26,10 @@ from .permute import seq_to_head, head_to_seq
 from .attention import (doc_starts, doc_ends, attention_forward, attention_backward,
                         bwd_preprocess, attention_rows, attention_kv_cols)
 from .layer import ulysses_layer_forward, ulysses_layer_backward
-from .projection import qkv_projection, out_projection
+from .projection import qkv_projection, out_projection, qkv_projection_backward, out_projection_backward
 
 __all__ = ["widen_bf16", "seq_to_head", "head_to_seq", "doc_starts", "doc_ends",
            "attention_forward", "attention_backward", "bwd_preprocess",
            "attention_rows", "attention_kv_cols",
-           "ulysses_layer_forward", "ulysses_layer_backward", "qkv_projection", "out_projection"]
+           "ulysses_layer_forward", "ulysses_layer_backward", "qkv_projection", "out_projection",
+           "qkv_projection_backward", "out_projection_backward"]

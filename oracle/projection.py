@@ -34,3 +34,30 @@ def out_projection(o_seq: List[np.ndarray], w_o: np.ndarray) -> List[np.ndarray]
         n = o.shape[0]
         out.append(np.asarray(o, np.float64).reshape(n, -1) @ np.asarray(w_o, np.float64).T)
     return out
+
+
+def qkv_projection_backward(x_seq: List[np.ndarray], w_qkv: np.ndarray, dq_seq, dk_seq, dv_seq):
+    """Gradient of qkv_projection: with g_t = [dq_t | dk_t | dv_t] (each head's d
+    values in head order), dx_t = g_t W_qkv and dW_qkv = sum_t g_t^T x_t.
+    Returns (dx_seq list [N/P, hidden], dW_qkv)."""
+    w = np.asarray(w_qkv, np.float64)
+    dx, dw = [], np.zeros_like(w)
+    for x, dq, dk, dv in zip(x_seq, dq_seq, dk_seq, dv_seq):
+        n = x.shape[0]
+        g = np.concatenate([np.asarray(t, np.float64).reshape(n, -1) for t in (dq, dk, dv)], axis=1)
+        dx.append(g @ w)
+        dw += g.T @ np.asarray(x, np.float64)
+    return dx, dw
+
+
+def out_projection_backward(o_seq: List[np.ndarray], w_o: np.ndarray, dy_seq: List[np.ndarray]):
+    """Gradient of out_projection: do_t = dy_t W_o (reshaped to [H, d]) and
+    dW_o = sum_t dy_t^T o_t. Returns (do_seq list [N/P, H, d], dW_o)."""
+    w = np.asarray(w_o, np.float64)
+    do, dw = [], np.zeros_like(w)
+    for o, dy in zip(o_seq, dy_seq):
+        n = o.shape[0]
+        dy = np.asarray(dy, np.float64)
+        do.append((dy @ w).reshape(o.shape))
+        dw += dy.T @ np.asarray(o, np.float64).reshape(n, -1)
+    return do, dw

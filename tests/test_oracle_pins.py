@@ -420,3 +420,62 @@ def test_projection_planted_transpose_is_caught():
     wrong = x @ w
     right = np.array([_brute_matvec(r, w) for r in x])
     assert not np.allclose(wrong, right, atol=1e-6)
+
+
+def test_projection_gradients_match_directional_derivatives():
+    """The projections are linear, so for L = sum_t <y_t, g_t> the change of L
+    along any direction E of an input or weight equals <gradient, E> exactly
+    (up to fp64 rounding): pins both backward formulas, including which side
+    of W each product takes and the head order of g."""
+    import oracle
+    rng = np.random.Generator(np.random.PCG64(75))
+    P, n, hidden, H, H_kv, d = 2, 3, 6, 4, 2, 2
+    x = [rng.standard_normal((n, hidden)) for _ in range(P)]
+    w = rng.standard_normal(((H + 2 * H_kv) * d, hidden))
+    gq = [rng.standard_normal((n, H, d)) for _ in range(P)]
+    gk = [rng.standard_normal((n, H_kv, d)) for _ in range(P)]
+    gv = [rng.standard_normal((n, H_kv, d)) for _ in range(P)]
+
+    def L(xs, ws):
+        q, k, v = oracle.qkv_projection(xs, ws, H, H_kv, d)
+        return sum(np.sum(a * b) for t, g in ((q, gq), (k, gk), (v, gv)) for a, b in zip(t, g))
+
+    dx, dw = oracle.qkv_projection_backward(x, w, gq, gk, gv)
+    Ew = rng.standard_normal(w.shape)
+    Ex = [rng.standard_normal(a.shape) for a in x]
+    eps = 1.0                       # exact for a linear map
+    assert abs((L(x, w + eps * Ew) - L(x, w)) - np.sum(dw * Ew)) < 1e-9
+    assert abs((L([a + eps * e for a, e in zip(x, Ex)], w) - L(x, w)) -
+               sum(np.sum(a * e) for a, e in zip(dx, Ex))) < 1e-9
+
+    o = [rng.standard_normal((n, H, d)) for _ in range(P)]
+    wo = rng.standard_normal((hidden, H * d))
+    gy = [rng.standard_normal((n, hidden)) for _ in range(P)]
+
+    def Lo(os_, ws):
+        return sum(np.sum(a * b) for a, b in zip(oracle.out_projection(os_, ws), gy))
+
+    do, dwo = oracle.out_projection_backward(o, wo, gy)
+    Ewo = rng.standard_normal(wo.shape)
+    Eo = [rng.standard_normal(a.shape) for a in o]
+    assert abs((Lo(o, wo + Ewo) - Lo(o, wo)) - np.sum(dwo * Ewo)) < 1e-9
+    assert abs((Lo([a + e for a, e in zip(o, Eo)], wo) - Lo(o, wo)) - sum(np.sum(a * e) for a, e in zip(do, Eo))) < 1e-9
+
+
+def test_projection_gradients_brute_force():
+    import math
+    import oracle
+    rng = np.random.Generator(np.random.PCG64(76))
+    n, hidden, H, d = 2, 3, 2, 2
+    o = [rng.standard_normal((n, H, d))]
+    wo = rng.standard_normal((hidden, H * d))
+    gy = [rng.standard_normal((n, hidden))]
+    do, dwo = oracle.out_projection_backward(o, wo, gy)
+    for t in range(n):
+        for f in range(H * d):
+            want = math.fsum(gy[0][t, k] * wo[k, f] for k in range(hidden))
+            assert abs(do[0].reshape(n, -1)[t, f] - want) < 1e-12
+    for k in range(hidden):
+        for f in range(H * d):
+            want = math.fsum(gy[0][t, k] * o[0].reshape(n, -1)[t, f] for t in range(n))
+            assert abs(dwo[k, f] - want) < 1e-12

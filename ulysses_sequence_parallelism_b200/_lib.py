@@ -36,6 +36,8 @@ _SIGS = {
     "ulysses_a2a_head_to_seq_frag": [_v, _v, _v, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _i, _i, _v],
     "ulysses_qkv_proj_seq_to_head": [_vpp, _v, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _i, _v],
     "ulysses_out_proj_head_to_seq": [_vpp, _v, _vpp, _i64, _i, _i, _i, _i, _i, _v],
+    "ulysses_out_proj_bwd": [_vpp, _v, _vpp, _vpp, _v, _i64, _i, _i, _i, _i, _i, _v],
+    "ulysses_qkv_proj_bwd": [_vpp, _v, _vpp, _vpp, _vpp, _vpp, _v, _i64, _i, _i, _i, _i, _i, _v],
     "ulysses_attn_fwd": [_vpp, _vpp, _vpp, _vpp, _fpp, _i64, _i, _i, _i, _i, _v, _i, _i, ctypes.c_float, _i,
                          _i, _i, _v],
     "ulysses_attn_bwd_workspace_size": [_i64, _i, _i, _i, _i, _i],

@@ -182,7 +182,14 @@ uly_status ulysses_qkv_proj_seq_to_head(const void* const* x_seq, const void* w_
   if (!ranks_ok(x_seq, 0, P) || !aligned16(w_qkv) || !ranks_ok(cv(q_head), 0, P) || !ranks_ok(cv(k_head), 0, P) ||
       !ranks_ok(cv(v_head), 0, P))
     return ULY_ERR_INVALID_ARG;
-  return from_cuda(uly::launch_proj(0, x_seq, w_qkv, q_head, k_head, v_head, N, P, H, H_kv, d, hidden, stream));
+  const void* wq[1] = {w_qkv};
+  uly::ProjGemm g{};
+  g.a_src = 0; g.b_src = 2; g.out_kind = 0; g.tok_m = 1;
+  g.a_bufs[0] = x_seq; g.a_ntensors = 1; g.a_seq_cols = hidden;
+  g.b_bufs[0] = wq; g.b_ntensors = 1; g.b_plain_rows = (H + 2 * H_kv) * d; g.b_plain_cols = hidden;
+  for (int r = 0; r < P; ++r) { g.out[0][r] = q_head[r]; g.out[1][r] = k_head[r]; g.out[2][r] = v_head[r]; }
+  g.N = N; g.P = P; g.K = hidden; g.n_out = (H + 2 * H_kv) * d; g.H = H; g.H_kv = H_kv; g.d = d;
+  return from_cuda(uly::launch_proj_gemm(g, stream));
 }
 
 uly_status ulysses_out_proj_head_to_seq(const void* const* o_head, const void* w_o, void* const* y_seq, int64_t N,
@@ -191,7 +198,75 @@ uly_status ulysses_out_proj_head_to_seq(const void* const* o_head, const void* w
   if (st != ULY_OK) return st;
   if (!ranks_ok(o_head, 0, P) || !aligned16(w_o) || !ranks_ok(reinterpret_cast<const void* const*>(y_seq), 0, P))
     return ULY_ERR_INVALID_ARG;
-  return from_cuda(uly::launch_proj(1, o_head, w_o, y_seq, nullptr, nullptr, N, P, H, H_kv, d, hidden, stream));
+  const void* wo[1] = {w_o};
+  uly::ProjGemm g{};
+  g.a_src = 1; g.b_src = 2; g.out_kind = 1; g.tok_m = 1;
+  g.a_bufs[0] = o_head; g.a_ntensors = 1;
+  g.b_bufs[0] = wo; g.b_ntensors = 1; g.b_plain_rows = hidden; g.b_plain_cols = static_cast<int64_t>(H) * d;
+  for (int r = 0; r < P; ++r) g.out[0][r] = y_seq[r];
+  g.N = N; g.P = P; g.K = H * d; g.n_out = hidden; g.H = H; g.H_kv = H_kv; g.d = d;
+  return from_cuda(uly::launch_proj_gemm(g, stream));
+}
+
+uly_status ulysses_out_proj_bwd(const void* const* o_head, const void* w_o, const void* const* dy_seq,
+                                void* const* do_head, void* dw_o, int64_t N, int P, int H, int H_kv, int d,
+                                int hidden, cudaStream_t stream) {
+  uly_status st = check_proj(N, P, H, H_kv, d, hidden);
+  if (st != ULY_OK) return st;
+  if ((H * d) % 256 != 0) return ULY_ERR_UNSUPPORTED;
+  if (!ranks_ok(o_head, 0, P) || !aligned16(w_o) || !ranks_ok(dy_seq, 0, P) ||
+      !ranks_ok(reinterpret_cast<const void* const*>(do_head), 0, P) || !aligned16(dw_o))
+    return ULY_ERR_INVALID_ARG;
+  const void* wo[1] = {w_o};
+  // dO = dY W_o, written into the head shards
+  uly::ProjGemm g{};
+  g.a_src = 0; g.b_src = 3; g.out_kind = 0; g.tok_m = 1;
+  g.a_bufs[0] = dy_seq; g.a_ntensors = 1; g.a_seq_cols = hidden;
+  g.b_bufs[0] = wo; g.b_ntensors = 1; g.b_plain_rows = hidden; g.b_plain_cols = static_cast<int64_t>(H) * d;
+  for (int r = 0; r < P; ++r) g.out[0][r] = do_head[r];
+  g.N = N; g.P = P; g.K = hidden; g.n_out = H * d; g.H = H; g.H_kv = H_kv; g.d = d;
+  cudaError_t e = uly::launch_proj_gemm(g, stream);
+  if (e != cudaSuccess) return from_cuda(e);
+  // dW_o = dY^T O, O read from the head shards
+  uly::ProjGemm w{};
+  w.a_src = 4; w.b_src = 5; w.out_kind = 2; w.tok_m = 0;
+  w.a_bufs[0] = dy_seq; w.a_ntensors = 1; w.a_seq_cols = hidden;
+  w.b_bufs[0] = o_head; w.b_ntensors = 1;
+  w.out[0][0] = dw_o;
+  w.N = N; w.P = P; w.K = static_cast<int>(N); w.n_out = H * d; w.m_rows = hidden; w.H = H; w.H_kv = H_kv; w.d = d;
+  return from_cuda(uly::launch_proj_gemm(w, stream));
+}
+
+uly_status ulysses_qkv_proj_bwd(const void* const* x_seq, const void* w_qkv, const void* const* dq_head,
+                                const void* const* dk_head, const void* const* dv_head, void* const* dx_seq,
+                                void* dw_qkv, int64_t N, int P, int H, int H_kv, int d, int hidden,
+                                cudaStream_t stream) {
+  uly_status st = check_proj(N, P, H, H_kv, d, hidden);
+  if (st != ULY_OK) return st;
+  if (!ranks_ok(x_seq, 0, P) || !aligned16(w_qkv) || !ranks_ok(dq_head, 0, P) || !ranks_ok(dk_head, 0, P) ||
+      !ranks_ok(dv_head, 0, P) || !ranks_ok(reinterpret_cast<const void* const*>(dx_seq), 0, P) ||
+      !aligned16(dw_qkv))
+    return ULY_ERR_INVALID_ARG;
+  const void* wq[1] = {w_qkv};
+  const int n_feat = (H + 2 * H_kv) * d;
+  // dX = [dQ|dK|dV] W_qkv, gathered from the head shards, written into the sequence shards
+  uly::ProjGemm g{};
+  g.a_src = 1; g.b_src = 3; g.out_kind = 1; g.tok_m = 1;
+  g.a_bufs[0] = dq_head; g.a_bufs[1] = dk_head; g.a_bufs[2] = dv_head; g.a_ntensors = 3;
+  g.b_bufs[0] = wq; g.b_ntensors = 1; g.b_plain_rows = n_feat; g.b_plain_cols = hidden;
+  for (int r = 0; r < P; ++r) g.out[0][r] = dx_seq[r];
+  g.N = N; g.P = P; g.K = n_feat; g.n_out = hidden; g.H = H; g.H_kv = H_kv; g.d = d;
+  cudaError_t e = uly::launch_proj_gemm(g, stream);
+  if (e != cudaSuccess) return from_cuda(e);
+  // dW_qkv = [dQ|dK|dV]^T X
+  uly::ProjGemm w{};
+  w.a_src = 5; w.b_src = 4; w.out_kind = 2; w.tok_m = 0;
+  w.a_bufs[0] = dq_head; w.a_bufs[1] = dk_head; w.a_bufs[2] = dv_head; w.a_ntensors = 3;
+  w.b_bufs[0] = x_seq; w.b_ntensors = 1; w.b_seq_cols = hidden;
+  w.out[0][0] = dw_qkv;
+  w.N = N; w.P = P; w.K = static_cast<int>(N); w.n_out = hidden; w.m_rows = n_feat; w.H = H; w.H_kv = H_kv;
+  w.d = d;
+  return from_cuda(uly::launch_proj_gemm(w, stream));
 }
 
 uly_status ulysses_attn_fwd(const void* const* q_head, const void* const* k_head, const void* const* v_head,

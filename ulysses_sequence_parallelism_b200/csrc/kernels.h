@@ -47,12 +47,23 @@ cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void
                             const void* const* dO, void* const* dq, void* const* dk, void* const* dv,
                             void* workspace, int deterministic, cudaStream_t stream);
 
-// Projections with the all-to-alls folded in. mode 0: a_bufs = X sequence
-// shards [N/P, hidden], w = W_qkv [(H + 2 H_kv) d, hidden], out0/1/2 = Q/K/V
-// head shards of all P ranks. mode 1: a_bufs = O head shards [N, H/P, d],
-// w = W_o [hidden, H d], out0 = Y sequence shards [N/P, hidden].
-cudaError_t launch_proj(int mode, const void* const* a_bufs, const void* w, void* const* out0, void* const* out1,
-                        void* const* out2, int64_t N, int P, int H, int H_kv, int d, int hidden,
-                        cudaStream_t stream);
+// One projection GEMM (C = A B^T over a reduction of K, bf16 in, fp32
+// accumulate, bf16 out) with operand views that fold the Ulysses all-to-alls
+// into its loads and stores. Sources (proj_sm100.cu, enum Src): 0 SEQ_K,
+// 1 HEAD_K, 2 PLAIN_K, 3 PLAIN_MN, 4 SEQ_MN, 5 HEAD_MN; outputs: 0 head shards,
+// 1 sequence shards, 2 plain row-major matrix.
+struct ProjGemm {
+  int a_src, b_src, out_kind, tok_m;
+  const void* const* a_bufs[3];   // per tensor: P head shards, or P sequence shards ([0]), or {matrix} ([0][0])
+  int a_ntensors;
+  int64_t a_plain_rows, a_plain_cols, a_seq_cols;
+  const void* const* b_bufs[3];
+  int b_ntensors;
+  int64_t b_plain_rows, b_plain_cols, b_seq_cols;
+  void* out[3][16];               // per tensor and rank / shard, or out[0][0]
+  int64_t N;
+  int P, K, n_out, m_rows, H, H_kv, d;
+};
+cudaError_t launch_proj_gemm(const ProjGemm& g, cudaStream_t stream);
 
 }  // namespace uly
