@@ -57,11 +57,6 @@ ULY_DEV float4 ld_shared_f4(uint32_t addr) {
   return v;
 }
 
-ULY_DEV void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-               : "memory");
-}
 
 // ====================================================================== prep
 struct PrepArgs {

@@ -76,42 +76,9 @@ ULY_DEV int doc_end_of(const int32_t* __restrict__ cu, int num_seqs, int i, int 
   return e <= i ? i + 1 : (e > N ? N : e);
 }
 
-// ----------------------------------------------------------------- mma.sync helpers
+// ----------------------------------------------------------------- addresses
 ULY_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-ULY_DEV void cp_async_16(uint32_t smem, const void* gmem, bool pred) {
-  int sz = pred ? 16 : 0;  // src-size 0 zero-fills the 16 bytes
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem), "l"(gmem), "r"(sz));
-}
-ULY_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
-template <int N>
-ULY_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
-
-ULY_DEV void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-ULY_DEV void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-
-// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32 accumulate.
-ULY_DEV void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Byte offset of 16-byte chunk `chunk` of row `row` in a [rows][D] bf16 tile
-// whose 16-byte chunks are XOR-swizzled by (row & 7) (conflict-free ldmatrix).
-template <int D>
-ULY_DEV uint32_t swz(int row, int chunk) {
-  return static_cast<uint32_t>(row * (D * 2) + ((chunk ^ (row & 7)) << 4));
 }
 
 }  // namespace uly
