@@ -483,7 +483,8 @@ def main():
                         "shards, and the gradients of all three (no permute launches)"}
         if w.backward:
             dy_seq = [torch.randn_like(t, dtype=torch.float32).to(torch.bfloat16) for t in y_seq]
-            dw_o, dw_qkv = torch.empty_like(w_o), torch.empty_like(w_qkv)
+            dw_o = torch.empty(w_o.shape, dtype=torch.float32, device=dev)
+            dw_qkv = torch.empty(w_qkv.shape, dtype=torch.float32, device=dev)
             dx_seq = [torch.empty_like(t) for t in x_seq]
             obwd_ms = timed(lambda: U.ulysses_out_proj_bwd(L.o_h, w_o, dy_seq, L.do_h, dw_o, N, P, H, H_kv, d,
                                                            hidden))

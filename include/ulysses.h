@@ -161,9 +161,12 @@ ULY_API uly_status ulysses_out_proj_head_to_seq(
  *   W_qkv (sequence shards [N/P, hidden]: no head->seq permute of dQ, dK, dV),
  *   and dw_qkv = sum over all tokens of [dq|dk|dv]_t^T x_t
  *   ([(H + 2 H_kv) d, hidden]).
- * fp32 accumulation over the whole reduction, one bf16 rounding (RNE). Weight
- * gradients are written, not accumulated into. Shape rules as the forward
- * projections; ulysses_out_proj_bwd also needs H d % 256 == 0. */
+ * dO and dX: fp32 accumulation over the whole reduction, one bf16 rounding
+ * (RNE). dw_o and dw_qkv are fp32 (they sum over every token): the call
+ * zeroes them and adds the partial sums of 4096-token chunks into them (fp32
+ * additions in L2, so their low bits may differ run to run); they are not
+ * accumulated across calls. Shape rules as the forward projections;
+ * ulysses_out_proj_bwd also needs H d % 256 == 0. */
 ULY_API uly_status ulysses_out_proj_bwd(
     const void* const* o_head, const void* w_o, const void* const* dy_seq,
     void* const* do_head, void* dw_o,

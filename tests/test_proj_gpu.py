@@ -23,6 +23,7 @@ SHAPES = [
     (1024, 2, 8, 2, 128, 1024),
     (1024, 4, 8, 4, 64, 512),
     (384, 1, 4, 4, 64, 256),      # P = 1, three 128-row tiles, one 256-column tile per tensor group
+    (9216, 2, 4, 4, 64, 256),     # weight gradients over 3 token chunks (4096, 4096, 1024) added in fp32
 ]
 
 
@@ -92,7 +93,7 @@ def test_out_projection_backward(N, P, H, H_kv, d, hidden):
     oh = [_dev(t) for t in oracle.seq_to_head(workloads.seq_shards(o, P))]
     dys = [_dev(t) for t in workloads.seq_shards(dy, P)]
     doh = [torch.empty(N, H // P, d, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
-    dwo = torch.empty(hidden, H * d, dtype=torch.bfloat16, device="cuda")
+    dwo = torch.empty(hidden, H * d, dtype=torch.float32, device="cuda")
     U.ulysses_out_proj_bwd(oh, _dev(w_o), dys, doh, dwo, N, P, H, H_kv, d, hidden)
     torch.cuda.synchronize()
     assert U.ulysses_get_device_status() == (0, 0)
@@ -118,7 +119,7 @@ def test_qkv_projection_backward(N, P, H, H_kv, d, hidden):
     dqh, dkh, dvh = heads(dq), heads(dk), heads(dv)
     xs = [_dev(t) for t in workloads.seq_shards(x, P)]
     dxs = [torch.empty(N // P, hidden, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
-    dw = torch.empty((H + 2 * H_kv) * d, hidden, dtype=torch.bfloat16, device="cuda")
+    dw = torch.empty((H + 2 * H_kv) * d, hidden, dtype=torch.float32, device="cuda")
     U.ulysses_qkv_proj_bwd(xs, _dev(w_qkv), dqh, dkh, dvh, dxs, dw, N, P, H, H_kv, d, hidden)
     torch.cuda.synchronize()
     assert U.ulysses_get_device_status() == (0, 0)

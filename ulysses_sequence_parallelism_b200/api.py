@@ -117,19 +117,20 @@ def ulysses_out_proj_head_to_seq(o_head, w_o, y_seq, N, P, H, H_kv, d, hidden, s
 
 
 def ulysses_out_proj_bwd(o_head, w_o, dy_seq, do_head, dw_o, N, P, H, H_kv, d, hidden, stream=None):
-    """dO = dY W_o into the head shards; dW_o = sum_t dy_t^T o_t."""
+    """dO = dY W_o into the head shards; dW_o (fp32) = sum_t dy_t^T o_t."""
     code = lib().ulysses_out_proj_bwd(
-        _ptrs(o_head, P), _one(w_o), _ptrs(dy_seq, P), _ptrs(do_head, P), _one(dw_o), N, P, H, H_kv, d, hidden,
+        _ptrs(o_head, P), _one(w_o), _ptrs(dy_seq, P), _ptrs(do_head, P), _one(dw_o, torch.float32), N, P, H,
+        H_kv, d, hidden,
         _stream(stream))
     check("ulysses_out_proj_bwd", code)
 
 
 def ulysses_qkv_proj_bwd(x_seq, w_qkv, dq_head, dk_head, dv_head, dx_seq, dw_qkv, N, P, H, H_kv, d, hidden,
                          stream=None):
-    """dX = [dQ|dK|dV] W_qkv into the sequence shards; dW_qkv = sum_t g_t^T x_t."""
+    """dX = [dQ|dK|dV] W_qkv into the sequence shards; dW_qkv (fp32) = sum_t g_t^T x_t."""
     code = lib().ulysses_qkv_proj_bwd(
         _ptrs(x_seq, P), _one(w_qkv), _ptrs(dq_head, P), _ptrs(dk_head, P), _ptrs(dv_head, P), _ptrs(dx_seq, P),
-        _one(dw_qkv), N, P, H, H_kv, d, hidden, _stream(stream))
+        _one(dw_qkv, torch.float32), N, P, H, H_kv, d, hidden, _stream(stream))
     check("ulysses_qkv_proj_bwd", code)
 
 
@@ -282,15 +283,16 @@ class UlyssesLayer:
     def backward_projected(self, dy_seq: List[torch.Tensor], x_seq: List[torch.Tensor], w_qkv: torch.Tensor,
                            w_o: torch.Tensor):
         """Backward of forward_projected (call it after forward_projected on the
-        same layer): dY -> (dX sequence shards, dW_qkv, dW_o). dO goes straight
+        same layer): dY -> (dX sequence shards, dW_qkv, dW_o); weight
+        gradients in fp32. dO goes straight
         into the head shards and dX is gathered straight from the attention
         gradients' head shards: no permute runs."""
         if not self.backward_enabled or self.fused or self.frag or self.rank_sequential:
             raise ValueError("backward_projected runs on the plain all-ranks layer with backward buffers")
         N, P, H, H_kv, d = self.N, self.P, self.H, self.H_kv, self.d
         hidden = x_seq[0].shape[1]
-        dw_o = torch.empty_like(w_o)
-        dw_qkv = torch.empty_like(w_qkv)
+        dw_o = torch.empty(w_o.shape, dtype=torch.float32, device=w_o.device)
+        dw_qkv = torch.empty(w_qkv.shape, dtype=torch.float32, device=w_qkv.device)
         dx_seq = [torch.empty_like(x) for x in x_seq]
         ulysses_out_proj_bwd(self.o_h, w_o, dy_seq, self.do_h, dw_o, N, P, H, H_kv, d, hidden)
         ulysses_attn_bwd(self.q_h, self.k_h, self.v_h, self.o_h, self.lse, self.do_h, self.dq_h, self.dk_h,

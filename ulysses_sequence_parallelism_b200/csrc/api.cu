@@ -122,6 +122,11 @@ uly_status a2a_fragment(bool seq_to_head, const void* const* seq0, const void* c
   return from_cuda(uly::launch_permute_fragment(seq_to_head, src, dst, hx, f_lo, f_cnt, N, P, d, stream));
 }
 
+// Token chunk of the split-K weight-gradient GEMMs: the chunk's rows of both
+// operands (<= 4096 x 6144 bf16 + 4096 x 4096 at the Llama shapes) stay in L2
+// while every output tile that needs them runs.
+constexpr int kProjTokenChunk = 4096;
+
 uly_status check_proj(int64_t N, int P, int H, int H_kv, int d, int hidden) {
   uly_status st = check_shape(N, P, H, H_kv, d, 0, P);
   if (st != ULY_OK) return st;
@@ -227,9 +232,11 @@ uly_status ulysses_out_proj_bwd(const void* const* o_head, const void* w_o, cons
   g.N = N; g.P = P; g.K = hidden; g.n_out = H * d; g.H = H; g.H_kv = H_kv; g.d = d;
   cudaError_t e = uly::launch_proj_gemm(g, stream);
   if (e != cudaSuccess) return from_cuda(e);
-  // dW_o = dY^T O, O read from the head shards
+  // dW_o = dY^T O (fp32), O read from the head shards; split over token chunks
+  e = cudaMemsetAsync(dw_o, 0, static_cast<size_t>(hidden) * H * d * sizeof(float), stream);
+  if (e != cudaSuccess) return from_cuda(e);
   uly::ProjGemm w{};
-  w.a_src = 4; w.b_src = 5; w.out_kind = 2; w.tok_m = 0;
+  w.a_src = 4; w.b_src = 5; w.out_kind = 3; w.tok_m = 0; w.k_chunk = kProjTokenChunk;
   w.a_bufs[0] = dy_seq; w.a_ntensors = 1; w.a_seq_cols = hidden;
   w.b_bufs[0] = o_head; w.b_ntensors = 1;
   w.out[0][0] = dw_o;
@@ -258,9 +265,11 @@ uly_status ulysses_qkv_proj_bwd(const void* const* x_seq, const void* w_qkv, con
   g.N = N; g.P = P; g.K = n_feat; g.n_out = hidden; g.H = H; g.H_kv = H_kv; g.d = d;
   cudaError_t e = uly::launch_proj_gemm(g, stream);
   if (e != cudaSuccess) return from_cuda(e);
-  // dW_qkv = [dQ|dK|dV]^T X
+  // dW_qkv = [dQ|dK|dV]^T X (fp32); split over token chunks
+  e = cudaMemsetAsync(dw_qkv, 0, static_cast<size_t>(n_feat) * hidden * sizeof(float), stream);
+  if (e != cudaSuccess) return from_cuda(e);
   uly::ProjGemm w{};
-  w.a_src = 5; w.b_src = 4; w.out_kind = 2; w.tok_m = 0;
+  w.a_src = 5; w.b_src = 4; w.out_kind = 3; w.tok_m = 0; w.k_chunk = kProjTokenChunk;
   w.a_bufs[0] = dq_head; w.a_bufs[1] = dk_head; w.a_bufs[2] = dv_head; w.a_ntensors = 3;
   w.b_bufs[0] = x_seq; w.b_ntensors = 1; w.b_seq_cols = hidden;
   w.out[0][0] = dw_qkv;

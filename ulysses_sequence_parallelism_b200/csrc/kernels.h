@@ -51,9 +51,11 @@ cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void
 // accumulate, bf16 out) with operand views that fold the Ulysses all-to-alls
 // into its loads and stores. Sources (proj_sm100.cu, enum Src): 0 SEQ_K,
 // 1 HEAD_K, 2 PLAIN_K, 3 PLAIN_MN, 4 SEQ_MN, 5 HEAD_MN; outputs: 0 head shards,
-// 1 sequence shards, 2 plain row-major matrix.
+// 1 sequence shards, 2 plain row-major bf16 matrix, 3 plain row-major fp32
+// matrix added into (split-K chunks of k_chunk reduction elements).
 struct ProjGemm {
   int a_src, b_src, out_kind, tok_m;
+  int k_chunk;
   const void* const* a_bufs[3];   // per tensor: P head shards, or P sequence shards ([0]), or {matrix} ([0][0])
   int a_ntensors;
   int64_t a_plain_rows, a_plain_cols, a_seq_cols;

@@ -55,7 +55,7 @@ enum Src : int {
   SEQ_MN = 4,   // rows = features of sequence shards (contiguous), reduction = tokens
   HEAD_MN = 5,  // rows = features of head shards (contiguous), reduction = tokens
 };
-enum Out : int { OUT_HEADS = 0, OUT_SEQ = 1, OUT_PLAIN = 2 };
+enum Out : int { OUT_HEADS = 0, OUT_SEQ = 1, OUT_PLAIN = 2, OUT_PLAIN_F32_ADD = 3 };
 
 struct Layout {
   static constexpr uint32_t kA = BM * BK * 2;          // 16 KB
@@ -73,6 +73,7 @@ struct GemmArgs {
   RankPtrsMut out[3];             // OUT_HEADS: [tensor].p[rank]; OUT_SEQ: [0].p[shard]; OUT_PLAIN: [0].p[0]
   int a_src, b_src, out_kind, a_mn, b_mn;
   int tok_m;                      // 1: output rows are tokens (tile = shard, row); 0: rows are features
+  int k_chunk;                    // > 0: blockIdx.z takes reduction range [z*k_chunk, +k_chunk) (split-K)
   int n_loc, P, K, n_out, H, H_kv, d;
   int m_tiles;                    // tok_m: row tiles per shard
 };
@@ -146,7 +147,14 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(const __grid_constant
   } else {
     m0 = blockIdx.y * BM;                                // first output feature row
   }
-  const int KT = a.K / BK;
+  // Reduction steps of this CTA: all of K, or one split-K chunk of it. With
+  // the split index slowest in the grid, the CTAs resident together share
+  // one chunk of the token-long operands, which then stays in L2.
+  int kt0 = 0, KT = a.K / BK;
+  if (a.k_chunk > 0) {
+    kt0 = blockIdx.z * (a.k_chunk / BK);
+    KT = min(a.K / BK - kt0, a.k_chunk / BK);
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i) mbar_init(bars + 8u * i, 1);
@@ -169,8 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(const __grid_constant
       if (!mbar_wait_warp(empty(s), ((kt / NS) & 1) ^ 1, kErrProj, 0x100 + s)) break;
       const uint32_t st = sbase + s * L::kStage;
       mbar_arrive_expect_tx_w(full(s), L::kStage);
-      load_slab(a, a.a_src, a.ta, st, BM, m0, p, s0, kt * BK, full(s));
-      load_slab(a, a.b_src, a.tb, st + L::kA, BN, n0, p, s0, kt * BK, full(s));
+      load_slab(a, a.a_src, a.ta, st, BM, m0, p, s0, (kt0 + kt) * BK, full(s));
+      load_slab(a, a.b_src, a.tb, st + L::kA, BN, n0, p, s0, (kt0 + kt) * BK, full(s));
     }
     for (int k = kt > NS ? kt - NS : 0; k < kt; ++k)
       mbar_wait_drain_w(full(k % NS), (k / NS) & 1, kErrProj, 0x1F0);
@@ -209,11 +217,22 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(const __grid_constant
         uint32_t v[32];
         tmem_ld32(tmem + loff + c * 32, v);
         tmem_wait_ld();
+        const int f = n0 + c * 32;                       // first output column of this chunk (inside one head)
+        if (a.out_kind == OUT_PLAIN_F32_ADD) {
+          // fp32 partial sum of this split-K chunk, added in L2
+          float* dstf = static_cast<float*>(a.out[0].p[0]) + static_cast<int64_t>(m0 + row) * a.n_out + f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dstf + 4 * e),
+                         "f"(__uint_as_float(v[4 * e])), "f"(__uint_as_float(v[4 * e + 1])),
+                         "f"(__uint_as_float(v[4 * e + 2])), "f"(__uint_as_float(v[4 * e + 3]))
+                         : "memory");
+          continue;
+        }
         uint4 o4[4];
         uint32_t* ow = reinterpret_cast<uint32_t*>(o4);
 #pragma unroll
         for (int e = 0; e < 16; ++e) ow[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-        const int f = n0 + c * 32;                       // first output column of this chunk (inside one head)
         __nv_bfloat16* dst;
         if (a.out_kind == OUT_HEADS) {
           int tn, q, col, hl;
@@ -273,6 +292,7 @@ cudaError_t launch_proj_gemm(const ProjGemm& g, cudaStream_t stream) {
   a->a_mn = (g.a_src == PLAIN_MN || g.a_src == SEQ_MN || g.a_src == HEAD_MN) ? 1 : 0;
   a->b_mn = (g.b_src == PLAIN_MN || g.b_src == SEQ_MN || g.b_src == HEAD_MN) ? 1 : 0;
   a->tok_m = g.tok_m;
+  a->k_chunk = g.k_chunk;
   a->n_loc = static_cast<int>(g.N / g.P);
   a->P = g.P;
   a->K = g.K;
@@ -294,7 +314,8 @@ cudaError_t launch_proj_gemm(const ProjGemm& g, cudaStream_t stream) {
     for (int r = 0; r < kMaxRanks; ++r) a->out[t].p[r] = g.out[t][r];
   cudaError_t e = cudaFuncSetAttribute(proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout::kAlloc);
   if (e == cudaSuccess) {
-    dim3 grid(g.n_out / BN, g.tok_m ? g.P * a->m_tiles : g.m_rows / BM);
+    const int splits = g.k_chunk > 0 ? (g.K + g.k_chunk - 1) / g.k_chunk : 1;
+    dim3 grid(g.n_out / BN, g.tok_m ? g.P * a->m_tiles : g.m_rows / BM, splits);
     proj_kernel<<<grid, kThreads, Layout::kAlloc, stream>>>(*a);
     e = cudaGetLastError();
   }
