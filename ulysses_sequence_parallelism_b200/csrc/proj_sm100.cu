@@ -91,42 +91,42 @@ ULY_DEV void feature_loc(const GemmArgs& a, int f, int& tensor, int& rank, int& 
   col = (head - rank * hl) * a.d + c;
 }
 
-// Issue the loads of one 64-deep slab of a tile of `rows` rows starting at r0
+// Issue the loads of one 64-deep slab of a tile of ROWS rows starting at r0
 // (tokens: shard p / row s0 / global t0) into dst.
-ULY_DEV void load_slab(const GemmArgs& a, int src, const CUtensorMap (*maps)[kMaxRanks], uint32_t dst, int rows,
-                       int r0, int p, int s0, int k0, uint32_t bar) {
-  switch (src) {
-    case SEQ_K:
-      tma_load_2d_w(dst, &maps[0][p], bar, k0, s0);
-      break;
-    case HEAD_K: {
+template <int SRC, int ROWS>
+ULY_DEV void load_slab(const GemmArgs& a, const CUtensorMap (*maps)[kMaxRanks], uint32_t dst, int r0, int p, int s0,
+                       int k0, uint32_t bar) {
+  if constexpr (SRC == SEQ_K) {
+    tma_load_2d_w(dst, &maps[0][p], bar, k0, s0);
+  } else if constexpr (SRC == HEAD_K) {
+    int t, q, x, hl;
+    feature_loc(a, k0, t, q, x, hl);
+    tma_load_2d_w(dst, &maps[t][q], bar, x, p * a.n_loc + s0);
+  } else if constexpr (SRC == PLAIN_K) {
+    tma_load_2d_w(dst, &maps[0][0], bar, k0, r0);
+  } else if constexpr (SRC == PLAIN_MN) {
+#pragma unroll
+    for (int i = 0; i < ROWS / 64; ++i) tma_load_2d_w(dst + 8192u * i, &maps[0][0], bar, r0 + 64 * i, k0);
+  } else if constexpr (SRC == SEQ_MN) {
+    const int sh = k0 / a.n_loc;
+#pragma unroll
+    for (int i = 0; i < ROWS / 64; ++i)
+      tma_load_2d_w(dst + 8192u * i, &maps[0][sh], bar, r0 + 64 * i, k0 - sh * a.n_loc);
+  } else {   // HEAD_MN
+#pragma unroll
+    for (int i = 0; i < ROWS / 64; ++i) {
       int t, q, x, hl;
-      feature_loc(a, k0, t, q, x, hl);
-      tma_load_2d_w(dst, &maps[t][q], bar, x, p * a.n_loc + s0);
-      break;
-    }
-    case PLAIN_K:
-      tma_load_2d_w(dst, &maps[0][0], bar, k0, r0);
-      break;
-    case PLAIN_MN:
-      for (int i = 0; i < rows / 64; ++i) tma_load_2d_w(dst + 8192u * i, &maps[0][0], bar, r0 + 64 * i, k0);
-      break;
-    case SEQ_MN: {
-      const int sh = k0 / a.n_loc;
-      for (int i = 0; i < rows / 64; ++i)
-        tma_load_2d_w(dst + 8192u * i, &maps[0][sh], bar, r0 + 64 * i, k0 - sh * a.n_loc);
-      break;
-    }
-    default: {   // HEAD_MN
-      for (int i = 0; i < rows / 64; ++i) {
-        int t, q, x, hl;
-        feature_loc(a, r0 + 64 * i, t, q, x, hl);
-        tma_load_2d_w(dst + 8192u * i, &maps[t][q], bar, x, k0);
-      }
+      feature_loc(a, r0 + 64 * i, t, q, x, hl);
+      tma_load_2d_w(dst + 8192u * i, &maps[t][q], bar, x, k0);
     }
   }
 }
 
+__host__ __device__ constexpr bool mn_major(int src) { return src == PLAIN_MN || src == SEQ_MN || src == HEAD_MN; }
+
+// One instantiation per (A view, B view, output) in use: every view and
+// descriptor constant is known at compile time.
+template <int ASRC, int BSRC, int OUTK>
 __global__ void __launch_bounds__(kThreads, 1) proj_kernel(const __grid_constant__ GemmArgs a) {
   using L = Layout;
   extern __shared__ uint8_t smem_raw[];
@@ -177,8 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(const __grid_constant
       if (!mbar_wait_warp(empty(s), ((kt / NS) & 1) ^ 1, kErrProj, 0x100 + s)) break;
       const uint32_t st = sbase + s * L::kStage;
       mbar_arrive_expect_tx_w(full(s), L::kStage);
-      load_slab(a, a.a_src, a.ta, st, BM, m0, p, s0, (kt0 + kt) * BK, full(s));
-      load_slab(a, a.b_src, a.tb, st + L::kA, BN, n0, p, s0, (kt0 + kt) * BK, full(s));
+      load_slab<ASRC, BM>(a, a.ta, st, m0, p, s0, (kt0 + kt) * BK, full(s));
+      load_slab<BSRC, BN>(a, a.tb, st + L::kA, n0, p, s0, (kt0 + kt) * BK, full(s));
     }
     for (int k = kt > NS ? kt - NS : 0; k < kt; ++k)
       mbar_wait_drain_w(full(k % NS), (k / NS) & 1, kErrProj, 0x1F0);
@@ -187,10 +187,11 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(const __grid_constant
     // ------------------------------------------------------------ MMA issuer
     // K-major tile: one 128-byte-swizzled box, K step = 32 bytes along the row.
     // M/N-major tile: 64-element atoms 8 KB apart (LBO), K step = 16 rows = 2 KB.
-    const uint32_t idesc = idesc_bf16_f32(BM, BN, a.a_mn, a.b_mn);
-    const uint64_t dA0 = smem_desc_sw128(sbase, a.a_mn ? 8192 : 16, 1024);
-    const uint64_t dB0 = smem_desc_sw128(sbase + L::kA, a.b_mn ? 8192 : 16, 1024);
-    const uint32_t ka = a.a_mn ? 2048 : 32, kb = a.b_mn ? 2048 : 32;
+    constexpr bool AMN = mn_major(ASRC), BMN = mn_major(BSRC);
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, AMN ? 1 : 0, BMN ? 1 : 0);
+    const uint64_t dA0 = smem_desc_sw128(sbase, AMN ? 8192 : 16, 1024);
+    const uint64_t dB0 = smem_desc_sw128(sbase + L::kA, BMN ? 8192 : 16, 1024);
+    constexpr uint32_t ka = AMN ? 2048 : 32, kb = BMN ? 2048 : 32;
     for (int kt = 0; kt < KT; ++kt) {
       const int s = kt % NS;
       if (!mbar_wait_warp(full(s), (kt / NS) & 1, kErrProj, 0x200 + s)) break;
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(const __grid_constant
         tmem_ld32(tmem + loff + c * 32, v);
         tmem_wait_ld();
         const int f = n0 + c * 32;                       // first output column of this chunk (inside one head)
-        if (a.out_kind == OUT_PLAIN_F32_ADD) {
+        if constexpr (OUTK == OUT_PLAIN_F32_ADD) {
           // fp32 partial sum of this split-K chunk, added in L2
           float* dstf = static_cast<float*>(a.out[0].p[0]) + static_cast<int64_t>(m0 + row) * a.n_out + f;
 #pragma unroll
@@ -234,11 +235,11 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(const __grid_constant
 #pragma unroll
         for (int e = 0; e < 16; ++e) ow[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
         __nv_bfloat16* dst;
-        if (a.out_kind == OUT_HEADS) {
+        if constexpr (OUTK == OUT_HEADS) {
           int tn, q, col, hl;
           feature_loc(a, f, tn, q, col, hl);
           dst = static_cast<__nv_bfloat16*>(a.out[tn].p[q]) + t * hl * a.d + col;
-        } else if (a.out_kind == OUT_SEQ) {
+        } else if constexpr (OUTK == OUT_SEQ) {
           dst = static_cast<__nv_bfloat16*>(a.out[0].p[p]) + static_cast<int64_t>(s0 + row) * a.n_out + f;
         } else {
           dst = static_cast<__nv_bfloat16*>(a.out[0].p[0]) + static_cast<int64_t>(m0 + row) * a.n_out + f;
@@ -312,11 +313,22 @@ cudaError_t launch_proj_gemm(const ProjGemm& g, cudaStream_t stream) {
   }
   for (int t = 0; t < 3; ++t)
     for (int r = 0; r < kMaxRanks; ++r) a->out[t].p[r] = g.out[t][r];
-  cudaError_t e = cudaFuncSetAttribute(proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout::kAlloc);
+  // the (A view, B view, output) combinations the entry points use
+  void (*kern)(GemmArgs) = nullptr;
+  if (g.a_src == SEQ_K && g.b_src == PLAIN_K && g.out_kind == OUT_HEADS) kern = proj_kernel<SEQ_K, PLAIN_K, OUT_HEADS>;
+  else if (g.a_src == HEAD_K && g.b_src == PLAIN_K && g.out_kind == OUT_SEQ) kern = proj_kernel<HEAD_K, PLAIN_K, OUT_SEQ>;
+  else if (g.a_src == SEQ_K && g.b_src == PLAIN_MN && g.out_kind == OUT_HEADS) kern = proj_kernel<SEQ_K, PLAIN_MN, OUT_HEADS>;
+  else if (g.a_src == SEQ_MN && g.b_src == HEAD_MN && g.out_kind == OUT_PLAIN_F32_ADD)
+    kern = proj_kernel<SEQ_MN, HEAD_MN, OUT_PLAIN_F32_ADD>;
+  else if (g.a_src == HEAD_K && g.b_src == PLAIN_MN && g.out_kind == OUT_SEQ) kern = proj_kernel<HEAD_K, PLAIN_MN, OUT_SEQ>;
+  else if (g.a_src == HEAD_MN && g.b_src == SEQ_MN && g.out_kind == OUT_PLAIN_F32_ADD)
+    kern = proj_kernel<HEAD_MN, SEQ_MN, OUT_PLAIN_F32_ADD>;
+  cudaError_t e = kern == nullptr ? cudaErrorInvalidValue : cudaSuccess;
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout::kAlloc);
   if (e == cudaSuccess) {
     const int splits = g.k_chunk > 0 ? (g.K + g.k_chunk - 1) / g.k_chunk : 1;
     dim3 grid(g.n_out / BN, g.tok_m ? g.P * a->m_tiles : g.m_rows / BM, splits);
-    proj_kernel<<<grid, kThreads, Layout::kAlloc, stream>>>(*a);
+    kern<<<grid, kThreads, Layout::kAlloc, stream>>>(*a);
     e = cudaGetLastError();
   }
   delete a;
