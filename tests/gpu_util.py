@@ -38,6 +38,12 @@ def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
     return np.where(ax > 0, np.exp2(e - 8), 0.0)
 
 
+# Below this magnitude a correctly rounded bf16 value is at most 2^-6 = 0.0156
+# off the exact one, so the raw bound MAX_ABS is attainable there. From 8 up a
+# bf16 step is 2^-4 and storage alone can miss 2e-2 by up to 2^-5.
+BIG_REF = 8.0
+
+
 def err_stats(gpu: np.ndarray, ref: np.ndarray):
     e = gpu - ref
     ma = float(np.max(np.abs(e))) if e.size else 0.0
@@ -47,22 +53,31 @@ def err_stats(gpu: np.ndarray, ref: np.ndarray):
 
 
 def assert_close(name, gpu, ref, max_abs=MAX_ABS, rel_rms=REL_RMS):
-    """Parity bar for bf16 results: relative RMS error <= rel_rms, and max
-    absolute error <= max_abs beyond the bf16 output's own half-ulp rounding
-    (an exact result stored in bf16 is already up to 2^-6 off at |x| in [4, 8),
-    2^-5 at [8, 16); the bar applies to the error the arithmetic adds)."""
+    """Parity bar for bf16 results against the fp64 oracle:
+      - relative RMS error <= rel_rms over the whole tensor;
+      - raw |gpu - ref| <= max_abs for every element with |ref| < 8;
+      - for elements with |ref| >= 8 only, where a correctly rounded bf16
+        value can already be 2^-5 off, the error beyond bf16's own half-ulp
+        rounding of ref must be <= max_abs.
+    Returns (raw max abs error, rel RMS, number of elements with |ref| >= 8)."""
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
     ma, rr = err_stats(gpu, ref)
-    excess = np.abs(gpu - ref) - bf16_half_ulp(ref)
-    mx = float(np.max(excess)) if excess.size else 0.0
-    if not (mx <= max_abs and rr <= rel_rms):
-        i = np.unravel_index(int(np.argmax(excess)), excess.shape)
-        big = int(np.sum(np.abs(ref) >= 4.0))
+    err = np.abs(gpu - ref)
+    big = np.abs(ref) >= BIG_REF
+    n_big = int(np.sum(big))
+    small_err = np.where(big, 0.0, err)
+    big_excess = np.where(big, err - bf16_half_ulp(ref), 0.0)
+    ms = float(np.max(small_err)) if err.size else 0.0
+    mb = float(np.max(big_excess)) if err.size else 0.0
+    if not (ms <= max_abs and mb <= max_abs and rr <= rel_rms):
+        worst = np.maximum(small_err, big_excess)
+        i = np.unravel_index(int(np.argmax(worst)), worst.shape)
         raise AssertionError(
-            f"{name}: max_abs {ma:.3e}, beyond half-ulp {mx:.3e} (<= {max_abs}), rel_rms {rr:.3e} (<= {rel_rms}); "
-            f"worst at {i}: gpu {gpu[i]:.6f} ref {ref[i]:.6f}; {big} elements with |ref| >= 4")
-    return ma, rr
+            f"{name}: raw max_abs {ma:.3e} (|ref|<8: {ms:.3e} <= {max_abs}; |ref|>=8 beyond half-ulp: {mb:.3e}), "
+            f"rel_rms {rr:.3e} (<= {rel_rms}); worst at {i}: gpu {gpu[i]:.6f} ref {ref[i]:.6f}; "
+            f"{n_big} elements with |ref| >= 8")
+    return ma, rr, n_big
 
 
 def sample_rows(N: int, P: int, cu_seqlens, count: int, seed: int = 0, tile: int = 128):

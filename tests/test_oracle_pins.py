@@ -479,3 +479,27 @@ def test_projection_gradients_brute_force():
         for f in range(H * d):
             want = math.fsum(gy[0][t, k] * o[0].reshape(n, -1)[t, f] for t in range(n))
             assert abs(dwo[k, f] - want) < 1e-12
+
+
+def test_widen_bf16_is_exact_on_every_bit_pattern():
+    """bf16 -> fp64 widening against torch's own bf16 -> float64 conversion on
+    all 65,536 bit patterns (finite values equal exactly; +-inf and NaN land in
+    the same classes), a few values fixed by the format (1, -2, the largest
+    finite value, the smallest subnormal), and the round trip through the
+    input generator's float32 -> bf16 rounding."""
+    import torch
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.widen_bf16(bits)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    fin = np.isfinite(ref)
+    assert fin.sum() == 65536 - 2 * 128                   # exponent field all ones: 2 signs x 128 mantissas
+    assert np.array_equal(ours[fin], ref[fin])
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+    assert np.array_equal(np.isposinf(ours), np.isposinf(ref)) and np.array_equal(np.isneginf(ours), np.isneginf(ref))
+    w = lambda b: float(oracle.widen_bf16(np.array([b], dtype=np.uint16))[0])
+    assert w(0x3F80) == 1.0 and w(0xC000) == -2.0 and w(0x0000) == 0.0
+    assert w(0x7F7F) == (2.0 - 2.0 ** -7) * 2.0 ** 127
+    assert w(0x0001) == 2.0 ** -133
+    assert w(0x3F81) == 1.0 + 2.0 ** -7                   # one bf16 step above 1 (7 stored mantissa bits)
+    back = workloads.round_to_bf16_bits(ours[fin].astype(np.float32))
+    assert np.array_equal(back, bits[fin])

@@ -23,7 +23,7 @@ __all__ = [
     "ulysses_selftest_bounded_wait", "ulysses_attn_fwd_seq", "ulysses_attn_bwd_seq", "UlyssesLayer",
     "HostPipeline", "ulysses_a2a_seq_to_head_frag", "ulysses_a2a_head_to_seq_frag",
     "ulysses_qkv_proj_seq_to_head", "ulysses_out_proj_head_to_seq", "ulysses_out_proj_bwd",
-    "ulysses_qkv_proj_bwd",
+    "ulysses_qkv_proj_bwd", "ulysses_a2a_pack", "ulysses_a2a_unpack",
 ]
 
 
@@ -99,6 +99,27 @@ def ulysses_a2a_head_to_seq_frag(x0_frag, x1_frag, x2_frag, x0_seq, x1_seq, x2_s
         _one(x0_frag), _one(x1_frag), _one(x2_frag), _ptrs(x0_seq, P), _ptrs(x1_seq, P), _ptrs(x2_seq, P),
         N, P, H, H_kv, d, head_lo, num_heads, _stream(stream))
     check("ulysses_a2a_head_to_seq_frag", code)
+
+
+def ulysses_a2a_pack(x0_seq, x1_seq, x2_seq, x0_send, x1_send, x2_send, N, P, H, H_kv, d, head_lo=0,
+                     num_heads=None, stream=None):
+    """One rank's sequence shards -> per-destination chunks [P, N/P, f, d] of
+    the head chunk [head_lo, head_lo + f) of every rank (for an all-to-all
+    between processes)."""
+    code = lib().ulysses_a2a_pack(
+        _one(x0_seq), _one(x1_seq), _one(x2_seq), _one(x0_send), _one(x1_send), _one(x2_send), N, P, H, H_kv, d,
+        head_lo, H // P if num_heads is None else num_heads, _stream(stream))
+    check("ulysses_a2a_pack", code)
+
+
+def ulysses_a2a_unpack(x0_recv, x1_recv, x2_recv, x0_seq, x1_seq, x2_seq, N, P, H, H_kv, d, head_lo=0,
+                       num_heads=None, stream=None):
+    """Inverse of ulysses_a2a_pack: received chunks [P, N/P, f, d] -> the
+    chunk's head columns of this rank's sequence shards."""
+    code = lib().ulysses_a2a_unpack(
+        _one(x0_recv), _one(x1_recv), _one(x2_recv), _one(x0_seq), _one(x1_seq), _one(x2_seq), N, P, H, H_kv, d,
+        head_lo, H // P if num_heads is None else num_heads, _stream(stream))
+    check("ulysses_a2a_unpack", code)
 
 
 def ulysses_qkv_proj_seq_to_head(x_seq, w_qkv, q_head, k_head, v_head, N, P, H, H_kv, d, hidden, stream=None):
@@ -247,7 +268,9 @@ class UlyssesLayer:
             nb = 0
         mk = lambda hx: [torch.empty(N, hx // P, d, dtype=bf, device=device) for _ in range(nb)]
         self.q_h, self.k_h, self.v_h, self.o_h = mk(H), mk(H_kv), mk(H_kv), mk(H)
-        self.lse = [torch.empty(H // P, N, dtype=f32, device=device) for _ in range(P if (fused or self.frag) else nb)]
+        # LSE of every rank is kept (it is what a backward needs; [H/P, N] fp32 per
+        # rank is small next to the head shards), also when ranks run one by one.
+        self.lse = [torch.empty(H // P, N, dtype=f32, device=device) for _ in range(P)]
         self.backward_enabled = backward and not rank_sequential
         if self.frag:
             f, fk = self.frag, self.frag // g
@@ -340,7 +363,7 @@ class UlyssesLayer:
                 rb = lambda b: self._rank_bufs(b, r)
                 ulysses_a2a_seq_to_head(q_seq, k_seq, v_seq, rb(self.q_h), rb(self.k_h), rb(self.v_h), N, P, H,
                                         H_kv, d, self.cu, rank_lo=r, rank_hi=r + 1)
-                ulysses_attn_fwd(rb(self.q_h), rb(self.k_h), rb(self.v_h), rb(self.o_h), rb(self.lse), N, P, H,
+                ulysses_attn_fwd(rb(self.q_h), rb(self.k_h), rb(self.v_h), rb(self.o_h), self.lse, N, P, H,
                                  H_kv, d, self.cu, self.max_seqlen, self.scale, rank_lo=r, rank_hi=r + 1)
                 ulysses_a2a_head_to_seq(rb(self.o_h), None, None, o_seq, None, None, N, P, H, H_kv, d, self.cu,
                                         rank_lo=r, rank_hi=r + 1)

@@ -44,8 +44,12 @@ extern "C" uly_status ulysses_attn_bwd_noalloc(
     const float* const* lse_head, const void* const* do_head, void* const* dq_head, void* const* dk_head,
     void* const* dv_head, int64_t N, int P, int H, int H_kv, int d, const int32_t* cu_seqlens, int num_seqs,
     int max_seqlen, float softmax_scale, int rank_lo, int rank_hi, cudaStream_t stream) {
+  // The shape check first, so a shape that ulysses_attn_bwd rejects gets the
+  // same status here (INVALID_ARG or UNSUPPORTED), before the size test.
+  const uly_status st = check_shape(N, P, H, H_kv, d, rank_lo, rank_hi);
+  if (st != ULY_OK) return st;
   const size_t need = ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, 1);
-  if (need == 0) return ULY_ERR_INVALID_ARG;                        // invalid shape
+  if (need == 0) return ULY_ERR_INVALID_ARG;
   if (need > uly::noalloc::kScratchBytes) return ULY_ERR_UNSUPPORTED;  // beyond the fixed scratch
   void* scratch = nullptr;
   if (uly::noalloc::scratch_address(&scratch) != cudaSuccess) return ULY_ERR_CUDA;
