@@ -122,6 +122,42 @@ ULY_API uly_status ulysses_a2a_head_to_seq_frag(
     void* const* x0_seq, void* const* x1_seq, void* const* x2_seq,
     int64_t N, int P, int H, int H_kv, int d, int head_lo, int num_heads, cudaStream_t stream);
 
+/* Pack / unpack for the exchange between processes (one process per GPU, each
+ * holding ONE rank's sequence shards; the all-to-all itself is a collective
+ * such as NCCL's). The method's first all-to-all sends, from every rank, each
+ * token's slice for every other rank's heads, so that each rank then holds
+ * the whole sequence for its own heads; the second undoes it
+ * (theaicatchup.com, "How Does Ulysses Sequence Parallelism Actually Work?";
+ * the Spanish note on contenidos2-1ml.pages.dev, "¿Qué cambia en la
+ * práctica…?", wants NVLink for this exchange).
+ * Sizes are those of the whole layer (N tokens in all, P ranks; this rank holds
+ * n = N/P). A head chunk [head_lo, head_lo + num_heads) inside every rank's H/P
+ * query heads (whole GQA groups: head_lo and num_heads multiples of
+ * g = H/H_kv, head_lo + num_heads <= H/P) and its key/value heads
+ * [head_lo/g, (head_lo + num_heads)/g) inside every rank's H_kv/P move; the
+ * chunk lets the exchange of one chunk overlap the attention of another.
+ * ulysses_a2a_pack: x0_seq [n, H, d] (x1_seq, x2_seq [n, H_kv, d]) of this
+ *   rank -> x0_send [P][n][f][d] (f = num_heads; f/g for slots 1, 2) with
+ *   x0_send[q][s][j] = x0_seq[s][q*H/P + head_lo + j]: chunk q is what rank q
+ *   must receive. After an all-to-all that delivers chunk q to rank q (in
+ *   source-rank order), each rank's receive buffer IS its [N, f, d] head
+ *   fragment (token p*n + s came from rank p), ready for ulysses_attn_fwd /
+ *   ulysses_attn_bwd with P = 1, H = f, H_kv = f/g.
+ * ulysses_a2a_unpack: the inverse, x0_recv [P][n][f][d] -> the chunk's head
+ *   columns of x0_seq (other columns untouched). The attention output [N, f, d]
+ *   of a rank is already [P][n][f][d] and is sent as is.
+ * x1/x2 may be NULL (both sides). Bit copies; pointers 16-byte aligned;
+ * caller-owned; asynchronous on `stream`. ULY_ERR_INVALID_ARG for a bad chunk
+ * or pointer, ULY_ERR_UNSUPPORTED beyond H*d <= 16384. */
+ULY_API uly_status ulysses_a2a_pack(
+    const void* x0_seq, const void* x1_seq, const void* x2_seq,
+    void* x0_send, void* x1_send, void* x2_send,
+    int64_t N, int P, int H, int H_kv, int d, int head_lo, int num_heads, cudaStream_t stream);
+ULY_API uly_status ulysses_a2a_unpack(
+    const void* x0_recv, const void* x1_recv, const void* x2_recv,
+    void* x0_seq, void* x1_seq, void* x2_seq,
+    int64_t N, int P, int H, int H_kv, int d, int head_lo, int num_heads, cudaStream_t stream);
+
 /* The projections on either side of the exchange, with the all-to-alls folded
  * into the GEMMs (each rank projects its own tokens before the first
  * all-to-all and its own shard after the second: theaicatchup.com, "How Does
@@ -239,7 +275,10 @@ ULY_API size_t ulysses_attn_bwd_workspace_size(int64_t N, int P, int H, int H_kv
  * sums dQ in fp32 with vector reductions in L2 (about 5/7 of the tensor work);
  * dK and dV are the same bits as the two-pass path, dQ agrees to fp32 rounding
  * but its low bits may differ between runs. With d == 64 both settings run
- * the two-pass kernels. */
+ * the two-pass kernels, and so does deterministic == 0 on a device where the
+ * one-pass kernel's shared-memory layout would not fit (see
+ * ulysses_attn_bwd_onepass_layout_fits); that choice is made on the host and
+ * never turns into an error status. */
 ULY_API uly_status ulysses_attn_bwd(
     const void* const* q_head, const void* const* k_head, const void* const* v_head,
     const void* const* o_head, const float* const* lse_head, const void* const* do_head,
@@ -307,6 +346,15 @@ ULY_API uly_status ulysses_get_device_status(cudaStream_t stream, uint32_t* deta
  * the default). Waits that drain a CTA before it exits always keep the default
  * cap. Synchronous; applies to the current device. */
 ULY_API void ulysses_set_wait_limit(uint32_t iters);
+
+/* Host-side selection rule of the backward (no CUDA call): returns 1 if the
+ * one-pass kernel's shared-memory layout fits when its dynamic shared memory
+ * starts `dyn_smem_offset` bytes into the CTA's shared window (the per-block
+ * reserved shared memory plus the kernel's static shared memory), else 0.
+ * ulysses_attn_bwd with deterministic = 0 applies this rule to the current
+ * device once and runs the two-pass kernels when it returns 0 (same dK/dV
+ * bits; dQ equal up to the order of its fp32 sums) instead of failing. */
+ULY_API int ulysses_attn_bwd_onepass_layout_fits(uint32_t dyn_smem_offset);
 
 /* Test hook: launches one tiny kernel on `stream` that waits, bounded, on an
  * mbarrier nothing arrives on (the same wait routine the attention kernels use),

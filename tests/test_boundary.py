@@ -167,3 +167,39 @@ def test_projection_entry_points_validate_before_launch(L):
                                           None) == 1
     assert L.ulysses_out_proj_head_to_seq(_arr([GOOD, 0]), w, p, 512, P, 8, 2, 128, 1024, None) == 1
     assert L.ulysses_out_proj_head_to_seq(p, w, p, 512, P, 8, 2, 128, 0, None) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(d=96), dict(d=256), dict(P=17, N=17 * 64, H=17, H_kv=17), dict(N=1023),
+                                dict(H_kv=3), dict(lo=2, hi=2)])
+def test_noalloc_returns_the_same_status_as_the_workspace_call(L, kw):
+    """Shapes the backward rejects get the same status from both entry points
+    (nothing is launched: validation fails first)."""
+    a = dict(N=1024, P=4, H=16, H_kv=4, d=128, lo=0, hi=None)
+    a.update(kw)
+    P = a["P"]
+    hi = P if a["hi"] is None else a["hi"]
+    fake = (ctypes.c_void_p * P)(*([0x10000] * P))
+    pp = ctypes.cast(fake, ctypes.POINTER(ctypes.c_void_p))
+    ws = ctypes.c_void_p(0x10000)
+    ref = L.ulysses_attn_bwd(pp, pp, pp, pp, pp, pp, pp, pp, pp, a["N"], P, a["H"], a["H_kv"], a["d"], None, 0, 0,
+                             0.0, 1, ws, 1 << 40, a["lo"], hi, None)
+    got = L.ulysses_attn_bwd_noalloc(pp, pp, pp, pp, pp, pp, pp, pp, pp, a["N"], P, a["H"], a["H_kv"], a["d"], None,
+                                     0, 0, 0.0, a["lo"], hi, None)
+    assert ref != 0
+    assert got == ref, (kw, got, ref)
+
+
+def test_onepass_backward_selection_rule(L):
+    """The backward picks the one-pass kernel only when its shared-memory
+    layout fits at the dynamic shared-memory offset the device gives it (else
+    it runs the two-pass kernels). Offsets at a 1024-byte boundary fit (the
+    case on sm_100: 1 KB reserved, no static shared memory); an offset just
+    past a boundary leaves the layout short by up to 1008 bytes and does not."""
+    f = L.ulysses_attn_bwd_onepass_layout_fits
+    assert f(0) == 1 and f(1024) == 1 and f(2048) == 1
+    assert f(1024 + 16) == 0 and f(1024 + 128) == 0
+    assert f(1024 - 16) == 1                      # 16 bytes of padding: fits
+    fits = [o for o in range(0, 2048, 16) if f(o)]
+    # the fitting offsets are those within a fixed distance below each boundary
+    pads = sorted({(1024 - o % 1024) % 1024 for o in fits})
+    assert pads == list(range(0, pads[-1] + 1, 16)) and pads[-1] < 1024

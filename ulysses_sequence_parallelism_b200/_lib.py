@@ -34,6 +34,8 @@ _SIGS = {
     "ulysses_a2a_head_to_seq": [_vpp, _vpp, _vpp, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _v, _i, _i, _i, _v],
     "ulysses_a2a_seq_to_head_frag": [_vpp, _vpp, _vpp, _v, _v, _v, _i64, _i, _i, _i, _i, _i, _i, _v],
     "ulysses_a2a_head_to_seq_frag": [_v, _v, _v, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _i, _i, _v],
+    "ulysses_a2a_pack": [_v, _v, _v, _v, _v, _v, _i64, _i, _i, _i, _i, _i, _i, _v],
+    "ulysses_a2a_unpack": [_v, _v, _v, _v, _v, _v, _i64, _i, _i, _i, _i, _i, _i, _v],
     "ulysses_qkv_proj_seq_to_head": [_vpp, _v, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _i, _v],
     "ulysses_out_proj_head_to_seq": [_vpp, _v, _vpp, _i64, _i, _i, _i, _i, _i, _v],
     "ulysses_out_proj_bwd": [_vpp, _v, _vpp, _vpp, _v, _i64, _i, _i, _i, _i, _i, _v],
@@ -47,6 +49,7 @@ _SIGS = {
     "ulysses_get_device_status": [_v, ctypes.POINTER(ctypes.c_uint32)],
     "ulysses_set_wait_limit": [ctypes.c_uint32],
     "ulysses_selftest_bounded_wait": [_v],
+    "ulysses_attn_bwd_onepass_layout_fits": [ctypes.c_uint32],
     "ulysses_attn_fwd_seq": [_vpp, _vpp, _vpp, _vpp, _fpp, _i64, _i, _i, _i, _i, _v, _i, _i, ctypes.c_float, _i,
                              _i, _i, _v],
     "ulysses_attn_bwd_seq": [_vpp, _vpp, _vpp, _vpp, _fpp, _vpp, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _v, _i,

@@ -122,6 +122,28 @@ uly_status a2a_fragment(bool seq_to_head, const void* const* seq0, const void* c
   return from_cuda(uly::launch_permute_fragment(seq_to_head, src, dst, hx, f_lo, f_cnt, N, P, d, stream));
 }
 
+// Pack/unpack for the multi-process exchange: one rank's shards and its
+// [P][N/P][f][d] chunk buffers; the head chunk is whole GQA groups.
+uly_status exchange(bool pack, const void* s0, const void* s1, const void* s2, void* d0, void* d1, void* d2,
+                    int64_t N, int P, int H, int H_kv, int d, int head_lo, int num_heads, cudaStream_t stream) {
+  uly_status st = check_shape(N, P, H, H_kv, d, 0, P);
+  if (st != ULY_OK) return st;
+  const int group = H / H_kv, hl = H / P;
+  if (num_heads < 1 || head_lo < 0 || head_lo + num_heads > hl) return ULY_ERR_INVALID_ARG;
+  if (head_lo % group != 0 || num_heads % group != 0) return ULY_ERR_INVALID_ARG;
+  if (s0 == nullptr || d0 == nullptr) return ULY_ERR_INVALID_ARG;
+  if ((s1 == nullptr) != (d1 == nullptr) || (s2 == nullptr) != (d2 == nullptr)) return ULY_ERR_INVALID_ARG;
+  const void* src[3] = {s0, s1, s2};
+  void* dst[3] = {d0, d1, d2};
+  for (int k = 0; k < 3; ++k)
+    if (src[k] != nullptr && (!aligned16(src[k]) || !aligned16(dst[k]))) return ULY_ERR_INVALID_ARG;
+  if (H * (d / 8) > uly::exchange_max_row_vecs()) return ULY_ERR_UNSUPPORTED;
+  const int hx[3] = {H, H_kv, H_kv};
+  const int lo[3] = {head_lo, head_lo / group, head_lo / group};
+  const int f[3] = {num_heads, num_heads / group, num_heads / group};
+  return from_cuda(uly::launch_exchange(pack, src, dst, hx, lo, f, N, P, d, stream));
+}
+
 // Token chunk of the split-K weight-gradient GEMMs: the chunk's rows of both
 // operands (<= 4096 x 6144 bf16 + 4096 x 4096 at the Llama shapes) stay in L2
 // while every output tile that needs them runs.
@@ -176,6 +198,20 @@ uly_status ulysses_a2a_head_to_seq_frag(const void* x0_frag, const void* x1_frag
   auto cv = [](void* const* p) { return reinterpret_cast<const void* const*>(p); };
   return a2a_fragment(false, cv(x0_seq), cv(x1_seq), cv(x2_seq), x0_frag, x1_frag, x2_frag, N, P, H, H_kv, d,
                       head_lo, num_heads, stream);
+}
+
+uly_status ulysses_a2a_pack(const void* x0_seq, const void* x1_seq, const void* x2_seq, void* x0_send,
+                            void* x1_send, void* x2_send, int64_t N, int P, int H, int H_kv, int d, int head_lo,
+                            int num_heads, cudaStream_t stream) {
+  return exchange(true, x0_seq, x1_seq, x2_seq, x0_send, x1_send, x2_send, N, P, H, H_kv, d, head_lo, num_heads,
+                  stream);
+}
+
+uly_status ulysses_a2a_unpack(const void* x0_recv, const void* x1_recv, const void* x2_recv, void* x0_seq,
+                              void* x1_seq, void* x2_seq, int64_t N, int P, int H, int H_kv, int d, int head_lo,
+                              int num_heads, cudaStream_t stream) {
+  return exchange(false, x0_recv, x1_recv, x2_recv, x0_seq, x1_seq, x2_seq, N, P, H, H_kv, d, head_lo, num_heads,
+                  stream);
 }
 
 uly_status ulysses_qkv_proj_seq_to_head(const void* const* x_seq, const void* w_qkv, void* const* q_head,
@@ -391,6 +427,10 @@ uly_status ulysses_get_device_status(cudaStream_t stream, uint32_t* detail) {
 }
 
 void ulysses_set_wait_limit(uint32_t iters) { cudaMemcpyToSymbol(uly::g_wait_limit, &iters, sizeof(iters)); }
+
+int ulysses_attn_bwd_onepass_layout_fits(uint32_t dyn_smem_offset) {
+  return uly::attn_bwd_onepass_layout_fits(dyn_smem_offset) ? 1 : 0;
+}
 
 uly_status ulysses_selftest_bounded_wait(cudaStream_t stream) {
   uly::selftest_wait_kernel<<<1, 32, 0, stream>>>();

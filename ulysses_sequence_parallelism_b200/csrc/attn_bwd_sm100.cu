@@ -824,6 +824,35 @@ cudaError_t launch_onepass(const AttnShape& s, const PrepArgs& pa, const DkdvArg
 
 bool attn_bwd_onepass(int d, int deterministic) { return !deterministic && d == bwd_sm100::onepass::D; }
 
+// The one-pass kernel uses all but a few hundred bytes of a CTA's shared memory
+// and aligns its tiles to 1024 bytes, so it fits only when its dynamic shared
+// memory starts close enough below a 1024-byte boundary. The dynamic area
+// starts after the per-block reserved shared memory and the kernel's static
+// shared memory: given that offset, does the layout fit?
+bool attn_bwd_onepass_layout_fits(uint32_t dyn_base_offset) {
+  const uint32_t pad = (1024u - dyn_base_offset % 1024u) % 1024u;
+  return pad + bwd_sm100::onepass::Layout::kUsed <= bwd_sm100::onepass::Layout::kAlloc;
+}
+
+// Whether the one-pass kernel's layout fits on the current device (looked up
+// once per device). When it does not, the backward runs the two-pass kernels
+// instead of returning an error: same dK/dV bits, dQ to summation order.
+bool attn_bwd_onepass_usable() {
+  constexpr int kMaxDev = 64;
+  static int cache[kMaxDev] = {};   // 0 unknown, 1 fits, 2 does not
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+  if (cache[dev] == 0) {
+    int reserved = 0;
+    cudaFuncAttributes fa;
+    if (cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, bwd_sm100::onepass::attn_bwd_onepass_kernel) != cudaSuccess)
+      return false;
+    cache[dev] = attn_bwd_onepass_layout_fits(static_cast<uint32_t>(reserved + fa.sharedSizeBytes)) ? 1 : 2;
+  }
+  return cache[dev] == 1;
+}
+
 size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d, int deterministic) {
   const int64_t npad = (N + bwd_sm100::TB - 1) / bwd_sm100::TB * bwd_sm100::TB;
   size_t bytes = 2 * static_cast<size_t>(P) * Hl * npad * sizeof(float);
@@ -861,7 +890,7 @@ cudaError_t launch_common(const AttnShape& s, PrepArgs& pa, DkdvArgs& ka, DqArgs
   ka.scale_log2 = qa.scale_log2 = s.scale * kLog2e;
   ka.rank_lo = qa.rank_lo = s.rank_lo;
   qa.num_m_tiles = (s.N + TB - 1) / TB;
-  if (attn_bwd_onepass(s.d, deterministic)) {
+  if (attn_bwd_onepass(s.d, deterministic) && attn_bwd_onepass_usable()) {
     ka.dqacc = Dv + static_cast<size_t>(s.P) * s.Hl * Npad;   // 512-byte aligned: Npad is a multiple of 128
     return launch_onepass(s, pa, ka, qa.dq, stream);
   }

@@ -27,6 +27,13 @@ cudaError_t launch_permute_fragment(bool seq_to_head, const void* const* src[3],
                                     const int hx[3], const int f_lo[3], const int f_cnt[3], int64_t N, int P, int d,
                                     cudaStream_t stream);
 
+// Pack (one rank's sequence shard -> per-destination chunks [P][N/P][f][d]) or
+// unpack (the inverse) of head chunk [lo[s], lo[s] + f[s]) inside every rank's
+// hx[s]/P heads, for up to three tensors (null src/dst: slot unused).
+int exchange_max_row_vecs();
+cudaError_t launch_exchange(bool pack, const void* const src[3], void* const dst[3], const int hx[3],
+                            const int lo[3], const int f[3], int64_t N, int P, int d, cudaStream_t stream);
+
 cudaError_t launch_attn_fwd(const AttnShape& s, const void* const* q, const void* const* k,
                             const void* const* v, void* const* o, float* const* lse, cudaStream_t stream);
 
@@ -42,6 +49,9 @@ cudaError_t launch_attn_bwd_seq(const AttnShape& s, const void* const* q_seq, co
 // deterministic == 0 with d == 128 selects the one-pass backward (fp32 dQ
 // accumulator in the workspace); everything else runs the two-pass kernels.
 size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d, int deterministic);
+// Whether the one-pass kernel's shared-memory layout fits when its dynamic
+// shared memory starts dyn_base_offset bytes into the CTA's shared window.
+bool attn_bwd_onepass_layout_fits(uint32_t dyn_base_offset);
 cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void* const* k,
                             const void* const* v, const void* const* o, const float* const* lse,
                             const void* const* dO, void* const* dq, void* const* dk, void* const* dv,
