@@ -11,6 +11,11 @@ Prints one JSON line (rank 0). Multi-GPU (torchrun): every rank runs its own
 independent layer (replicas; the path has no cross-GPU step on one GPU's
 emulated ranks), value = total tokens of all ranks / max-over-ranks time.
 
+--workload million times the rank-sequential forward (P = 8 virtual ranks one
+after another, N = 1,048,576); --all-workloads adds, under the key
+"workloads", one summary per other workload of the pages' 8K-1M range
+(tokens/s, attention TFLOP/s with roofline fractions, permute GB/s).
+
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload instead (rank 0 only).
 """
@@ -55,11 +60,14 @@ def kernel_source_hash(files):
     return h.hexdigest()
 
 
-def stored_traffic(workload, stage):
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+
+
+def stored_traffic(workload, stage, path=None):
     """DRAM bytes per call of `stage` from profiles/roofline_traffic.json, or
     None when they were taken on other kernel sources or another workload."""
     try:
-        with open(os.path.join(ROOT, "profiles", "roofline_traffic.json")) as f:
+        with open(path or TRAFFIC_FILE) as f:
             t = json.load(f)
         st = t[stage]
         if t.get("workload") != workload or st["source_sha256"] != kernel_source_hash(st["sources"]):
@@ -132,6 +140,128 @@ def aggregate_over_ranks(local_ms: float, tokens_per_rank: int, world: int, redu
     process group, `reduce_max` is an all-reduce(max) over ranks."""
     ms = reduce_max(local_ms) if (world > 1 and reduce_max is not None) else local_ms
     return ms, world * tokens_per_rank / (ms / 1e3)
+
+
+def device_inputs(w, dev, seed=0):
+    """Seeded synthetic inputs drawn on the device (fast at any size): the
+    workload's document lengths from its numpy recipe, then Q, K, V, dO as
+    N(0,1) x scale rounded to bf16 by a CUDA generator seeded with `seed`.
+    Used for timing only; parity tests draw with workloads.generate."""
+    import torch
+    cu = None
+    if w.varlen is not None:
+        rng = np.random.Generator(np.random.PCG64(seed))
+        cu = workloads.cu_seqlens_from_lengths(workloads.draw_doc_lengths(rng, w.N, *w.varlen))
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    n = w.N // w.P
+    mk = lambda hx, sc: [(torch.randn(n, hx, w.d, device=dev, generator=g) * sc).to(torch.bfloat16)
+                         for _ in range(w.P)]
+    out = {"cu_seqlens": cu, "q": mk(w.H, w.scale), "k": mk(w.H_kv, w.scale), "v": mk(w.H_kv, w.scale)}
+    if w.backward:
+        out["do"] = mk(w.H, 1.0)
+    return out
+
+
+def time_layer(U, w, dev, q, k, v, do, cu_np, steps, warmup, deterministic=False, barrier=None):
+    """Time `steps` layer steps of workload `w` (after `warmup` untimed ones)
+    stage by stage with CUDA events on the launching stream. All ranks at once,
+    or one rank after another for rank-sequential workloads (the stage times
+    are then summed over ranks). Returns the layer, the total ms, per-stage
+    mean ms lists and the kernel launch count per step."""
+    import torch
+    N, P, H, H_kv, d = w.N, w.P, w.H, w.H_kv, w.d
+    cu = None if cu_np is None else torch.tensor(cu_np, dtype=torch.int32, device=dev)
+    layer = U.UlyssesLayer(N, P, H, H_kv, d, device=dev, cu_seqlens=cu, backward=w.backward,
+                           rank_sequential=w.rank_sequential, deterministic=deterministic)
+    o = [torch.empty_like(x) for x in q]
+    if w.backward:
+        dq = [torch.empty_like(x) for x in q]
+        dk = [torch.empty_like(x) for x in k]
+        dv = [torch.empty_like(x) for x in v]
+    stream = torch.cuda.current_stream()
+    stages = ["qkv_s2h", "attn_fwd", "o_h2s"] + (["do_s2h", "attn_bwd", "dqkv_h2s"] if w.backward else [])
+    ranges = [(r, r + 1) for r in range(P)] if w.rank_sequential else [(0, P)]
+    L = layer
+
+    def bufs(b, lo, hi):
+        # all-ranks layers hold P head buffers; rank-sequential ones reuse one
+        return b if not w.rank_sequential else [b[0] if i == lo else None for i in range(P)]
+
+    def step(ev=None):
+        for ri, (lo, hi) in enumerate(ranges):
+            rec = (lambda i: ev[ri][i].record(stream)) if ev else (lambda i: None)
+            rec(0)
+            U.ulysses_a2a_seq_to_head(q, k, v, bufs(L.q_h, lo, hi), bufs(L.k_h, lo, hi), bufs(L.v_h, lo, hi), N, P,
+                                      H, H_kv, d, cu, rank_lo=lo, rank_hi=hi)
+            rec(1)
+            U.ulysses_attn_fwd(bufs(L.q_h, lo, hi), bufs(L.k_h, lo, hi), bufs(L.v_h, lo, hi), bufs(L.o_h, lo, hi),
+                               L.lse, N, P, H, H_kv, d, cu, rank_lo=lo, rank_hi=hi)
+            rec(2)
+            U.ulysses_a2a_head_to_seq(bufs(L.o_h, lo, hi), None, None, o, None, None, N, P, H, H_kv, d, cu,
+                                      rank_lo=lo, rank_hi=hi)
+            rec(3)
+            if w.backward:
+                U.ulysses_a2a_seq_to_head(do, None, None, L.do_h, None, None, N, P, H, H_kv, d, cu)
+                rec(4)
+                U.ulysses_attn_bwd(L.q_h, L.k_h, L.v_h, L.o_h, L.lse, L.do_h, L.dq_h, L.dk_h, L.dv_h, N, P, H, H_kv,
+                                   d, L.workspace, cu, deterministic=deterministic)
+                rec(5)
+                U.ulysses_a2a_head_to_seq(L.dq_h, L.dk_h, L.dv_h, dq, dk, dv, N, P, H, H_kv, d, cu)
+                rec(6)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    code, word = U.ulysses_get_device_status()
+    if code != 0:
+        raise SystemExit(f"{w.name}: device status {code} word {word:#x} after warm-up")
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in ranges]
+           for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if barrier is not None:
+        barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for s_ in range(steps):
+        step(evs[s_])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if barrier is not None:
+        barrier()
+    code, word = U.ulysses_get_device_status()
+    if code != 0:
+        raise SystemExit(f"{w.name}: device status {code} word {word:#x} after the timed steps")
+    stage_ms = {st: [sum(evs[s_][ri][i].elapsed_time(evs[s_][ri][i + 1]) for ri in range(len(ranges)))
+                     for s_ in range(steps)] for i, st in enumerate(stages)}
+    launches = len(ranges) * 3 + ((1 + 3 + 1) if w.backward else 0)
+    outs = {"o": o}
+    if w.backward:
+        outs.update(dq=dq, dk=dk, dv=dv)
+    return layer, t0.elapsed_time(t1), stage_ms, launches, outs
+
+
+def summarize(w, cu_np, total_ms, stage_ms, steps, peaks):
+    """Tokens/s, attention TFLOP/s and permute GB/s of one timed workload."""
+    f_fwd, f_bwd, pairs = flops(w, cu_np)
+    pb = permute_bytes(w)
+    mean = {st: sum(v_) / len(v_) for st, v_ in stage_ms.items()}
+    ms = total_ms / steps
+    out = {"workload": w.name, "N": w.N, "P": w.P, "pass": "fwd+bwd" if w.backward else "fwd",
+           "rank_sequential": w.rank_sequential, "docs": None if cu_np is None else int(len(cu_np) - 1),
+           "steps": steps, "ms_per_step": ms, "tokens_per_s": w.N / (ms / 1e3), "stage_ms_mean": mean,
+           "pairs": pairs, "attn_fwd_tflops": f_fwd / (mean["attn_fwd"] / 1e3) / 1e12,
+           "permute_gbs": {st: pb[st] / (mean[st] / 1e3) / 1e9 for st in pb if st in mean}}
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    out["attn_fwd_frac_of_burst"] = out["attn_fwd_tflops"] / burst
+    out["attn_fwd_frac_of_sustained"] = out["attn_fwd_tflops"] / sus
+    if w.backward:
+        out["attn_bwd_tflops"] = f_bwd / (mean["attn_bwd"] / 1e3) / 1e12
+        out["attn_bwd_frac_of_sustained"] = out["attn_bwd_tflops"] / sus
+    hp = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    out["permute_frac_of_hbm"] = {st: g / hp for st, g in out["permute_gbs"].items()}
+    return out
 
 
 def cpu_oracle_sample(w, inp, budget_s=20.0):
@@ -225,6 +355,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--deterministic", action="store_true",
                     help="time the two-pass backward (bit-reproducible dQ) instead of the one-pass one")
+    ap.add_argument("--all-workloads", action="store_true",
+                    help="also time llama8k, single64k, long96k and the million-token workload (key 'workloads')")
     ap.add_argument("--tokens", type=int, default=None,
                     help="draw the workload's recipe at a smaller total N (profiling captures)")
     args = ap.parse_args()
@@ -252,81 +384,36 @@ def main():
         if world > 1:
             dist.barrier()
 
-    inp = workloads.generate(w, seed=0)
-    cu_np = inp["cu_seqlens"]
-    cu = None if cu_np is None else torch.tensor(cu_np, dtype=torch.int32, device=dev)
+    inp = workloads.generate(w, seed=0) if not w.rank_sequential else None
     P, H, H_kv, d, N = w.P, w.H, w.H_kv, w.d, w.N
-    layer = U.UlyssesLayer(N, P, H, H_kv, d, device=dev, cu_seqlens=cu, backward=w.backward,
-                           rank_sequential=w.rank_sequential, deterministic=args.deterministic)
 
     def shards(x):
         n = N // P
         return [torch.from_numpy(x[p * n:(p + 1) * n].view(np.int16)).view(torch.bfloat16).to(dev) for p in range(P)]
 
-    q, k, v = shards(inp["q"]), shards(inp["k"]), shards(inp["v"])
-    do = shards(inp["do"]) if w.backward else None
-    o = [torch.empty_like(x) for x in q]
-    if w.backward:
-        dq = [torch.empty_like(x) for x in q]
-        dk = [torch.empty_like(x) for x in k]
-        dv = [torch.empty_like(x) for x in v]
+    if inp is not None:
+        cu_np = inp["cu_seqlens"]
+        q, k, v = shards(inp["q"]), shards(inp["k"]), shards(inp["v"])
+        do = shards(inp["do"]) if w.backward else None
+    else:
+        # rank-sequential (million-token) workload: seeded inputs drawn on the device
+        di = device_inputs(w, dev)
+        cu_np, q, k, v, do = di["cu_seqlens"], di["q"], di["k"], di["v"], di.get("do")
+    cu = None if cu_np is None else torch.tensor(cu_np, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
-
     f_fwd, f_bwd, pairs = flops(w, cu_np)
     pb = permute_bytes(w)
-    stages = ["qkv_s2h", "attn_fwd", "o_h2s"] + (["do_s2h", "attn_bwd", "dqkv_h2s"] if w.backward else [])
 
-    def step(ev=None):
-        """One layer step; ev: list of len(stages)+1 events to record between stages."""
-        L = layer
-        if ev: ev[0].record(stream)
-        U.ulysses_a2a_seq_to_head(q, k, v, L.q_h, L.k_h, L.v_h, N, P, H, H_kv, d, cu)
-        if ev: ev[1].record(stream)
-        U.ulysses_attn_fwd(L.q_h, L.k_h, L.v_h, L.o_h, L.lse, N, P, H, H_kv, d, cu)
-        if ev: ev[2].record(stream)
-        U.ulysses_a2a_head_to_seq(L.o_h, None, None, o, None, None, N, P, H, H_kv, d, cu)
-        if ev: ev[3].record(stream)
-        if w.backward:
-            U.ulysses_a2a_seq_to_head(do, None, None, L.do_h, None, None, N, P, H, H_kv, d, cu)
-            if ev: ev[4].record(stream)
-            U.ulysses_attn_bwd(L.q_h, L.k_h, L.v_h, L.o_h, L.lse, L.do_h, L.dq_h, L.dk_h, L.dv_h, N, P, H, H_kv, d,
-                               L.workspace, cu, deterministic=args.deterministic)
-            if ev: ev[5].record(stream)
-            U.ulysses_a2a_head_to_seq(L.dq_h, L.dk_h, L.dv_h, dq, dk, dv, N, P, H, H_kv, d, cu)
-            if ev: ev[6].record(stream)
-
-    if w.rank_sequential:
-        raise SystemExit("bench.py times all-rank workloads; the million-token workload is a parity case")
-
-    launches_per_step = 1 + 1 + 1 + ((1 + 3 + 1) if w.backward else 0)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    code, word = U.ulysses_get_device_status()
-    if code != 0:
-        raise SystemExit(f"device status {code} word {word:#x} after warm-up")
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    t_begin = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_begin.record(stream)
-    for s in range(args.steps):
-        step(evs[s])
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    barrier()
+    layer, total_ms, stage_ms, launches_per_step, outs = time_layer(
+        U, w, dev, q, k, v, do, cu_np, args.steps, args.warmup, deterministic=args.deterministic, barrier=barrier)
     clk = clocks.stop()
-    total_ms = t_begin.elapsed_time(t_end)
-    stage_ms = {st: [] for st in stages}
-    for s in range(args.steps):
-        for i, st in enumerate(stages):
-            stage_ms[st].append(evs[s][i].elapsed_time(evs[s][i + 1]))
+    o = outs["o"]
+    if w.backward:
+        dq, dk, dv = outs["dq"], outs["dk"], outs["dv"]
+
     def reduce_max(x):
         t = torch.tensor([x], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -341,6 +428,9 @@ def main():
     perm_gbs = {st: pb[st] / (mean[st] / 1e3) / 1e9 for st in pb if st in mean}
     detail = {"attn_fwd_tflops": fwd_tflops, "permute_gbs": perm_gbs,
               "stage_ms_mean": mean, "stage_ms_median": med, "pairs": pairs, "attn_fwd_flops": f_fwd}
+    if w.rank_sequential:
+        detail["note"] = (f"{P} virtual ranks one after another (seq->head, attention, head->seq per rank); "
+                          "stage times summed over ranks")
     if w.backward:
         detail["attn_bwd_tflops"] = f_bwd / (mean["attn_bwd"] / 1e3) / 1e12
         detail["attn_bwd_flops"] = f_bwd
@@ -479,8 +569,8 @@ def main():
         proj = {"hidden": hidden, "qkv_proj_ms": qkv_ms, "qkv_proj_tflops": f_qkv / (qkv_ms / 1e3) / 1e12,
                 "out_proj_ms": out_ms, "out_proj_tflops": f_out / (out_ms / 1e3) / 1e12,
                 "block_fwd_ms": blk_ms, "block_fwd_tokens_per_s": N / (blk_ms / 1e3),
-                "note": "block = QKV projection into head shards + attention + output projection from head "
-                        "shards, and the gradients of all three (no permute launches)"}
+                "note": "block_fwd = QKV projection into head shards + attention + output projection from head "
+                        "shards (forward only); block_fwd_bwd adds the gradients of all three; no permute launches"}
         if w.backward:
             dy_seq = [torch.randn_like(t, dtype=torch.float32).to(torch.bfloat16) for t in y_seq]
             dw_o = torch.empty(w_o.shape, dtype=torch.float32, device=dev)
@@ -506,7 +596,7 @@ def main():
     # HostPipeline: every step copies its inputs from pinned host memory and
     # reads its results back; copies of neighbouring steps overlap the kernels.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and inp is not None:
         pin = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
         n = N // P
         rows = lambda a: [pin(a[p * n:(p + 1) * n]) for p in range(P)]
@@ -542,7 +632,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_oracle_sample(w, inp, budget_s=20.0)
+        cb = cpu_oracle_sample(w, inp if inp is not None else workloads.generate(w, N=16384), budget_s=20.0)
         cpu = {k_: cb[k_] for k_ in ("value", "unit", "cores", "kind", "sample")}
 
     if rank == 0:
@@ -560,6 +650,33 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk, "detail": detail, "fused": fused, "head_fragment": frag, "projections": proj,
         }
+        if inp is None:
+            line["config"]["inputs"] = "seeded N(0,1) drawn on the device (torch CUDA generator, seed 0)"
+    # ---------------------------------------------------------------- the other workloads (opt-in)
+    # the pages' range, 8K to 1M tokens: one summary per workload, not the headline
+    if args.all_workloads:
+        extra = {}
+        del o, layer, outs
+        if w.backward:
+            del dq, dk, dv
+        torch.cuda.empty_cache()
+        for name in ("llama8k", "varlen64k", "single64k", "long96k", "million"):
+            if name == w.name:
+                continue
+            wx = workloads.get(name)
+            di = device_inputs(wx, dev)
+            steps_x = 1 if wx.rank_sequential else max(3, min(args.steps, 10))
+            warm_x = 1 if wx.rank_sequential else 3
+            _, tot, st_ms, _, _ = time_layer(U, wx, dev, di["q"], di["k"], di["v"], di.get("do"), di["cu_seqlens"],
+                                             steps_x, warm_x, deterministic=args.deterministic, barrier=barrier)
+            tot, _ = aggregate_over_ranks(tot, wx.N, world, reduce_max)
+            extra[name] = summarize(wx, di["cu_seqlens"], tot, st_ms, steps_x, peaks)
+            extra[name]["inputs"] = "seeded N(0,1) x scale drawn on the device (torch CUDA generator, seed 0)"
+            del di
+            torch.cuda.empty_cache()
+        if rank == 0:
+            line["workloads"] = extra
+    if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

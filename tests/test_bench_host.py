@@ -18,18 +18,35 @@ def _bench():
     return bench
 
 
-def test_stored_traffic_matches_current_sources():
+def _traffic_file(bench, tmp_path, workload="varlen64k"):
+    t = {"workload": workload}
+    for stage, files, b in (("attn_bwd", ["attn_bwd_sm100.cu", "common.cuh"], 123),
+                            ("attn_fwd", ["attn_fwd_sm100.cu", "sm100.cuh"], 456)):
+        t[stage] = {"bytes": b, "sources": files, "source_sha256": bench.kernel_source_hash(files)}
+    p = tmp_path / "traffic.json"
+    p.write_text(json.dumps(t))
+    return str(p)
+
+
+def test_stored_traffic_matches_current_sources(tmp_path):
     bench = _bench()
-    with open(os.path.join(ROOT, "profiles", "roofline_traffic.json")) as f:
-        t = json.load(f)
-    for stage in ("attn_bwd", "attn_fwd"):
-        assert bench.stored_traffic("varlen64k", stage) == t[stage]["bytes"]
-        assert bench.stored_traffic("single64k", stage) is None          # other workload
-    assert bench.stored_traffic("varlen64k", "no_such_stage") is None
+    p = _traffic_file(bench, tmp_path)
+    assert bench.stored_traffic("varlen64k", "attn_bwd", p) == 123
+    assert bench.stored_traffic("varlen64k", "attn_fwd", p) == 456
+    assert bench.stored_traffic("single64k", "attn_fwd", p) is None          # other workload
+    assert bench.stored_traffic("varlen64k", "no_such_stage", p) is None
 
 
 def test_stored_traffic_goes_null_when_a_source_changes(tmp_path, monkeypatch):
     bench = _bench()
-    real = bench.kernel_source_hash
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda files: "0" * 64 if files else real(files))
-    assert bench.stored_traffic("varlen64k", "attn_bwd") is None
+    p = _traffic_file(bench, tmp_path)
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda files: "0" * 64)
+    assert bench.stored_traffic("varlen64k", "attn_bwd", p) is None
+
+
+def test_committed_traffic_file_is_well_formed():
+    bench = _bench()
+    with open(bench.TRAFFIC_FILE) as f:
+        t = json.load(f)
+    for stage in ("attn_bwd", "attn_fwd"):
+        assert t[stage]["bytes"] > 0 and t[stage]["sources"] and len(t[stage]["source_sha256"]) == 64
