@@ -344,6 +344,105 @@ def run_reference(args, w):
     return 0
 
 
+def run_exchange(args, w):
+    """The real multi-process exchange: P = the number of processes, each
+    holding N/P tokens of the workload's sequence (the whole job processes N
+    tokens per step, so more GPUs means fewer tokens each: strong scaling).
+    A step is UlyssesDistLayer forward (+ backward): pack, NCCL all-to-all,
+    attention on the received head chunk, all-to-all back, unpack."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import ulysses_sequence_parallelism_b200 as U
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    if world == 1:
+        import socket
+        with socket.socket() as s_:
+            s_.bind(("127.0.0.1", 0))
+            os.environ.setdefault("MASTER_PORT", str(s_.getsockname()[1]))
+        os.environ.setdefault("RANK", "0")
+        os.environ.setdefault("WORLD_SIZE", "1")
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    N, H, H_kv, d = w.N, w.H, w.H_kv, w.d
+    if N % world or H % world or H_kv % world:
+        raise SystemExit(f"--exchange needs N, H, H_kv divisible by the {world} processes")
+    cu_np = None
+    if w.varlen is not None:
+        rng = np.random.Generator(np.random.PCG64(0))
+        cu_np = workloads.cu_seqlens_from_lengths(workloads.draw_doc_lengths(rng, N, *w.varlen))
+    cu = None if cu_np is None else torch.tensor(cu_np, dtype=torch.int32, device=dev)
+    n = N // world
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + rank)
+    mk = lambda hx, sc: (torch.randn(n, hx, d, device=dev, generator=g) * sc).to(torch.bfloat16)
+    q, k, v = mk(H, w.scale), mk(H_kv, w.scale), mk(H_kv, w.scale)
+    do = mk(H, 1.0) if w.backward else None
+    layer = U.UlyssesDistLayer(N, H, H_kv, d, device=dev, cu_seqlens=cu, backward=w.backward)
+    o = torch.empty_like(q)
+    if w.backward:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(q, k, v, o)
+        if w.backward:
+            layer.backward(do, dq, dk, dv)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    code, word = U.ulysses_get_device_status()
+    if code != 0:
+        raise SystemExit(f"device status {code} word {word:#x}")
+    t = torch.tensor([e0.elapsed_time(e1) / args.steps], device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    f_fwd, f_bwd, pairs = flops(w, cu_np)
+    shard = lambda hx: n * hx * d * 2
+    per_pass = 2 * shard(H) + 2 * shard(H_kv)                 # Q, K, V in + O out (forward)
+    sent = (world - 1) / world * (per_pass + (2 * shard(H) + 2 * shard(H_kv) if w.backward else 0))
+    line = {
+        "metric": "Ulysses layer tokens/s (fwd+bwd)" if w.backward else "Ulysses layer tokens/s (fwd)",
+        "value": N / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "N": N, "P": world, "H": H, "H_kv": H_kv, "d": d,
+                   "docs": None if cu_np is None else int(len(cu_np) - 1),
+                   "pass": "fwd+bwd" if w.backward else "fwd",
+                   "parallelism": f"Ulysses over {world} processes (NCCL all-to-all, "
+                                  f"{len(layer.plan.chunks)} head chunks)",
+                   "inputs": "seeded N(0,1) drawn on each rank's device"},
+        "exchange": {"bytes_sent_per_rank_per_step": sent, "chunks": len(layer.plan.chunks),
+                     "attn_tflops_whole_job": (f_fwd + (f_bwd if w.backward else 0)) / (ms / 1e3) / 1e12},
+        "clocks": clk,
+        # per chunk: pack, attention, unpack (+ backward: pack dO, three backward kernels, unpack)
+        "gpu_launches": len(layer.plan.chunks) * (3 + (5 if w.backward else 0)) * args.steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del layer
+    dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -353,8 +452,14 @@ def main():
     ap.add_argument("--workload", default="varlen64k", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layer-only", action="store_true",
+                    help="time only the layer step (no fused / fragment / projection / e2e / CPU extras); "
+                         "for profiler captures")
     ap.add_argument("--deterministic", action="store_true",
                     help="time the two-pass backward (bit-reproducible dQ) instead of the one-pass one")
+    ap.add_argument("--exchange", choices=["none", "nccl"], default="none",
+                    help="nccl: run the real multi-process exchange (P = number of processes) instead of "
+                         "independent replicas")
     ap.add_argument("--all-workloads", action="store_true",
                     help="also time llama8k, single64k, long96k and the million-token workload (key 'workloads')")
     ap.add_argument("--tokens", type=int, default=None,
@@ -366,6 +471,8 @@ def main():
         w = dataclasses.replace(w, N=args.tokens)
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.exchange == "nccl":
+        return run_exchange(args, w)
 
     import torch
     import torch.distributed as dist
@@ -435,6 +542,7 @@ def main():
         detail["attn_bwd_tflops"] = f_bwd / (mean["attn_bwd"] / 1e3) / 1e12
         detail["attn_bwd_flops"] = f_bwd
         detail["attn_bwd_mode"] = "two-pass (deterministic)" if args.deterministic else "one-pass (fp32 dQ reductions)"
+    if w.backward and not args.layer_only:
         # the other backward mode on the same buffers, for comparison (not part of the step)
         other = not args.deterministic
         L = layer
@@ -470,8 +578,10 @@ def main():
                 "frac": achieved / hp, "traffic": None, "peak_source": f"{peak_src} hbm_gbs"}
 
     # ---------------------------------------------------------------- fused layer (all-to-alls in the kernels)
+    if args.layer_only:
+        args.no_e2e = args.no_cpu_baseline = True
     fused = None
-    if w.backward and (N // P) % 128 == 0:
+    if w.backward and (N // P) % 128 == 0 and not args.layer_only:
         lf = U.UlyssesLayer(N, P, H, H_kv, d, device=dev, cu_seqlens=cu, fused=True,
                             deterministic=args.deterministic)
 
@@ -504,7 +614,7 @@ def main():
     # each rank processes its heads one GQA group at a time: same results, a
     # fraction of the full-sequence activation buffers
     frag = None
-    if w.backward:
+    if w.backward and not args.layer_only:
         g = H // H_kv
         lfr = U.UlyssesLayer(N, P, H, H_kv, d, device=dev, cu_seqlens=cu, head_fragment=g,
                              deterministic=args.deterministic)
@@ -539,7 +649,7 @@ def main():
     # QKV projection storing straight into the head shards and output projection
     # reading straight from them (hidden = H d, synthetic seeded weights)
     proj = None
-    if not w.rank_sequential and (N // P) % 128 == 0:
+    if not w.rank_sequential and (N // P) % 128 == 0 and not args.layer_only:
         hidden = H * d
         xb, wqb, wob = workloads.projection_inputs(N, H, H_kv, d, hidden, seed=1)
         tdev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)

@@ -72,6 +72,9 @@ CASES = [
     (384, 1, 8, 1, 128, [0, 129, 384]),               # P = 1, GQA 8:1
     (256, 4, 4, 4, 64, [0, 64, 65, 256]),             # P = H (one head per rank), doc of length 1
     (320, 4, 8, 4, 128, [0, 17, 100, 101, 240, 320]),  # GQA 2:1, many documents
+    # 16 heads x 16 row blocks = 256 forward work items: more than one per SM, so
+    # the persistent forward carries its pipelines from one item to the next
+    (4096, 2, 16, 4, 128, [0, 1, 700, 701, 2500, 4096]),
 ]
 
 

@@ -24,6 +24,7 @@ SHAPES = [
     (1024, 4, 8, 4, 64, 512),
     (384, 1, 4, 4, 64, 256),      # P = 1, three 128-row tiles, one 256-column tile per tensor group
     (9216, 2, 4, 4, 64, 256),     # weight gradients over 3 token chunks (4096, 4096, 1024) added in fp32
+    (1024, 4, 32, 8, 128, 4096),  # the Llama-3-8B layer at the hidden size the bench times (H d = 4096)
 ]
 
 
