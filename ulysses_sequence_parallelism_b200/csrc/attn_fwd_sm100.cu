@@ -34,8 +34,17 @@ using namespace sm100;
 constexpr int BM = 128;        // query rows per tile (two tiles per CTA)
 constexpr int BN = 128;        // keys per K/V block
 constexpr int NSTAGE = 4;      // K/V ring stages (K and V blocks alternate)
-constexpr int kThreads = 320;  // 8 softmax warps + TMA warp + MMA warp
+// Three warpgroups: two softmax warpgroups (warps 0-3, 4-7) and one holding
+// the TMA producer (warp 8), the MMA issuer (warp 9) and two idle warps. At
+// launch every thread gets 168 registers (3 warps per SM sub-partition share
+// its 16K registers); the TMA/MMA warpgroup then gives registers back
+// (setmaxnreg.dec to kRegsCtl) and the softmax warpgroups take them
+// (setmaxnreg.inc to kRegsSoftmax): 2*128*200 + 128*104 = 384*168, exactly the
+// launch's total, so every increase is covered.
+constexpr int kThreads = 384;
 constexpr int kTmaWarp = 8, kMmaWarp = 9;
+constexpr int kRegsSoftmax = 200, kRegsCtl = 104;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCtl <= kThreads * 168, "register split above the launch total");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O when the max grows by > 2^8
@@ -80,6 +89,7 @@ struct Layout {
 };
 
 ULY_DEV float u2f(uint32_t x) { return __uint_as_float(x); }
+
 ULY_DEV float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -144,6 +154,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
   const uint32_t tS[2] = {tmem, tmem + 128};
   const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
 
+  // Each role's code must sit inside the branch that changes its register
+  // count (the compiler applies the new limit to the code the change dominates).
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     {
@@ -287,7 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
       mbar_wait_drain_w(mma_done, 0, kErrFwd, 0x350);
     }
     __syncwarp();
+  }   // warps 10 and 11: nothing to do
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ------------------------------------------------------------ softmax / epilogue
     // Per-warp scalars (no runtime-indexed arrays: they would live in local memory).
     const int t = warp >> 2;
@@ -316,28 +332,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
         tmem_wait_ld();
         const int n0 = jb * BN;
         const bool need_mask = (n0 + BN - 1 > frow) || (n0 < max_start);
+        // Row max on the raw scores (the scale is positive, so it commutes with
+        // max); masked keys become -inf and give exactly 0 below.
+        if (need_mask) {
+          const int lo = st_i - n0, hi = i - n0;   // allowed columns: lo <= c <= hi
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c < lo || c > hi) v[c] = __float_as_uint(-INFINITY);
+        }
         float mx[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
-        if (need_mask) {
+        for (int e = 0; e < 8; ++e) mx[e] = max3f(u2f(v[2 * e]), u2f(v[2 * e + 1]), -INFINITY);
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const int key = n0 + c;
-            float x = u2f(v[c]) * sl2;
-            x = (key > i || key < st_i) ? -INFINITY : x;
-            v[c] = __float_as_uint(x);
-            mx[c & 7] = fmaxf(mx[c & 7], x);
-          }
-        } else {
+        for (int c = 16; c < BN; c += 16)
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const float x = u2f(v[c]) * sl2;
-            v[c] = __float_as_uint(x);
-            mx[c & 7] = fmaxf(mx[c & 7], x);
-          }
-        }
-        const float m_blk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          for (int e = 0; e < 8; ++e) mx[e] = max3f(mx[e], u2f(v[c + 2 * e]), u2f(v[c + 2 * e + 1]));
+        const float mraw = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+        const float m_blk = mraw * sl2;           // -inf stays -inf
         const float m_new = fmaxf(m_run, m_blk);
         // Rescale decision (warp-uniform: TMEM loads/stores are warp-collective).
         bool rescale = false;
@@ -350,15 +361,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
           l_run *= alpha;
           m_run = m_new;
         }
-        const float base = (m_run == -INFINITY) ? 0.f : m_run;
+        // p = 2^(s * scale*log2(e) - base): scale and subtraction in one packed
+        // FFMA per two keys, then one ex2 each; row sum with packed adds.
+        const float nbase = (m_run == -INFINITY) ? 0.f : -m_run;
         float rs[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) rs[e] = 0.f;
 #pragma unroll
         for (int c = 0; c < BN; c += 2) {
-          const float p0 = ex2_approx(u2f(v[c]) - base);
-          const float p1 = ex2_approx(u2f(v[c + 1]) - base);
-          rs[(c >> 1) & 7] += p0 + p1;
+          float x0, x1;
+          ffma2_sc(x0, x1, u2f(v[c]), u2f(v[c + 1]), sl2, nbase);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          const int e = (c >> 1) & 3;
+          fadd2_acc(rs[2 * e], rs[2 * e + 1], p0, p1);
           v[c / 2] = pack_bf16x2(p0, p1);
         }
         l_run += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));

@@ -44,6 +44,29 @@ ULY_DEV float ex2_approx(float x) {
   return y;
 }
 
+// Three-input fp32 max (one instruction on sm_100).
+ULY_DEV float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed fp32 pair arithmetic (sm_100 f32x2): two lanes of work per instruction.
+// (d0, d1) = (a0 * s + c, a1 * s + c)
+ULY_DEV void ffma2_sc(float& d0, float& d1, float a0, float a1, float s, float c) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\tmov.b64 c, {%5, %5};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(s), "f"(c));
+}
+// (acc0, acc1) += (a0, a1)
+ULY_DEV void fadd2_acc(float& acc0, float& acc1, float a0, float a1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(acc0), "=f"(acc1)
+      : "f"(acc0), "f"(acc1), "f"(a0), "f"(a1));
+}
+
 ULY_DEV uint32_t pack_bf16x2(float lo, float hi) {
   // cvt.rn.bf16x2.f32 d, a, b puts a in the upper half and b in the lower half.
   uint32_t r;
