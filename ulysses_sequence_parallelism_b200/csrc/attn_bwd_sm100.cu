@@ -796,7 +796,7 @@ cudaError_t launch_onepass(const AttnShape& s, const PrepArgs& pa, const DkdvArg
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, onepass::Layout::kAlloc);
     if (e != cudaSuccess) return e;
     dim3 grid(s.Hkvl * nranks, (s.N + TB - 1) / TB);
-    onepass::attn_bwd_onepass_kernel<<<grid, kThreads, onepass::Layout::kAlloc, stream>>>(ka);
+    onepass::attn_bwd_onepass_kernel<<<grid, onepass::kOpThreads, onepass::Layout::kAlloc, stream>>>(ka);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -11,8 +11,8 @@
 // One CTA owns two 128-row query tiles of one head (256 rows) and streams the
 // 128-key K/V blocks they need through a 4-stage shared-memory ring:
 //   warp 8      : TMA producer (Q tiles once, then K_j, V_j alternately)
-//   warp 9      : MMA issuer: S_t = Q_t K_j^T (SS, K-major both), then
-//                 O_t += P_t V_j (A = P from TMEM, B = V MN-major)
+//   warp 9      : MMA issuer: S_t = Q_t K_j^T (SS, K-major both, N = 128),
+//                 then O_t += P_t V_j (A = P from TMEM, B = V MN-major)
 //   warps 0-3/4-7: softmax of tile 0 / tile 1, one thread per row: reads its
 //                 S row from TMEM, online softmax in the log2 domain with fp32
 //                 statistics, writes P (bf16) back over S, rescales its O row
@@ -39,11 +39,11 @@ constexpr int NSTAGE = 4;      // K/V ring stages (K and V blocks alternate)
 // launch every thread gets 168 registers (3 warps per SM sub-partition share
 // its 16K registers); the TMA/MMA warpgroup then gives registers back
 // (setmaxnreg.dec to kRegsCtl) and the softmax warpgroups take them
-// (setmaxnreg.inc to kRegsSoftmax): 2*128*200 + 128*104 = 384*168, exactly the
+// (setmaxnreg.inc to kRegsSoftmax): 2*128*208 + 128*88 = 384*168, exactly the
 // launch's total, so every increase is covered.
 constexpr int kThreads = 384;
 constexpr int kTmaWarp = 8, kMmaWarp = 9;
-constexpr int kRegsSoftmax = 200, kRegsCtl = 104;
+constexpr int kRegsSoftmax = 208, kRegsCtl = 88;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCtl <= kThreads * 168, "register split above the launch total");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -208,12 +208,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    // Order per key block j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1). S is issued
-    // as two N=64 halves; P lives in S's columns [0,64), so the upper half
-    // (columns 64..127) goes out right behind PV(j) and only the lower half
-    // waits for PV(j) to have read P -- the wait is hidden behind the upper half.
+    // Order per key block j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1). P lives in
+    // S's columns [0, 64), so S(j+1) is issued once PV(j) has read P. One
+    // warp serves both tiles in this fixed order, which keeps the two tiles'
+    // softmax phases alternating instead of competing for the exponential
+    // unit (one issuing warp per tile measured 9 % slower).
     {
-      constexpr uint32_t idS = idesc_bf16_f32(BM, BN / 2, 0, 0);
+      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(BM, D, 0, 1);
       bool ok = true;
 #pragma unroll
@@ -224,15 +225,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
       const uint64_t dQ0 = smem_desc_sw128(sQ, 16, 1024);
       const uint64_t dRing0 = smem_desc_sw128(sRing, 16, 1024);
       const uint64_t dRingV0 = smem_desc_sw128(sRing, BN * 128, 1024);
-      auto issue_s_half = [&](int t, uint32_t kb, int half) {
+      // S_t = Q_t K^T over the whole 128-key block: N = 128 SS MMAs run at the
+      // full tensor rate (two N = 64 halves are shared-memory bound, 48 cycles
+      // per MMA instead of 32 per 64 columns).
+      auto issue_s = [&](int t, uint32_t kb) {
         const uint64_t qd = desc_adv(dQ0, t * L::kQTile);
-        const uint64_t kd = desc_adv(dRing0, kb - sRing + half * (64 * 128));
-        const uint32_t dst = tS[t] + half * 64;
+        const uint64_t kd = desc_adv(dRing0, kb - sRing);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off_q = (kk / 4) * (BM * 128) + (kk % 4) * 32;
           const uint32_t off_k = (kk / 4) * (BN * 128) + (kk % 4) * 32;
-          mma_ss_w(dst, desc_adv(qd, off_q), desc_adv(kd, off_k), idS, kk > 0 ? 1u : 0u);
+          mma_ss_w(tS[t], desc_adv(qd, off_q), desc_adv(kd, off_k), idS, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, uint32_t vb, int cnt) {
@@ -252,8 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (!part(t, jb_lo)) continue;
-            issue_s_half(t, sRing, 1);
-            issue_s_half(t, sRing, 0);
+            issue_s(t, sRing);
             mma_commit_w(s_full(t));
           }
           mma_commit_w(kv_empty(0));
@@ -279,16 +281,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
             issue_pv(t, vb, cnt[t]);
             mma_commit_w(pv_done(t));
             if (nxt) {
-              issue_s_half(t, kb, 1);
+              // S(j+1) overwrites the columns P(j) is read from: after PV(j)
               if (!mbar_wait_warp(pv_done(t), cnt[t] & 1, kErrFwd, 0x320 + t)) { ok = false; break; }
               tc_fence_after();
-              issue_s_half(t, kb, 0);
+              issue_s(t, kb);
               mma_commit_w(s_full(t));
             }
             ++cnt[t];
           } else if (nxt) {
-            issue_s_half(t, kb, 1);
-            issue_s_half(t, kb, 0);
+            issue_s(t, kb);
             mma_commit_w(s_full(t));
           }
         }
@@ -326,9 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100_kernel(const __gri
         if (!mbar_wait_warp(s_full(t), cnt & 1, kErrFwd, 0x400 + t)) { ok = false; break; }
         tc_fence_after();
         uint32_t v[BN];
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
-          tmem_ld32(tSt + lane_off + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
+        tmem_ld128(tSt + lane_off, v);
         tmem_wait_ld();
         const int n0 = jb * BN;
         const bool need_mask = (n0 + BN - 1 > frow) || (n0 < max_start);
