@@ -197,7 +197,7 @@ def test_onepass_backward_selection_rule(L):
     past a boundary leaves the layout short by up to 1008 bytes and does not."""
     f = L.ulysses_attn_bwd_onepass_layout_fits
     assert f(0) == 1 and f(1024) == 1 and f(2048) == 1
-    assert f(1024 + 16) == 0 and f(1024 + 128) == 0
+    assert f(1024 + 16) == 0 and f(1024 + 64) == 0
     assert f(1024 - 16) == 1                      # 16 bytes of padding: fits
     fits = [o for o in range(0, 2048, 16) if f(o)]
     # the fitting offsets are those within a fixed distance below each boundary

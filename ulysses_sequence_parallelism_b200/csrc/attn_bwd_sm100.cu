@@ -120,8 +120,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ P
 
 // ====================================================================== dK, dV
 struct DkdvArgs {
-  CUtensorMap tq[kMaxRanks];    // box 64 cols x SB rows
-  CUtensorMap tdo[kMaxRanks];   // box 64 cols x SB rows
+  CUtensorMap tq[kMaxRanks];    // box 64 cols x SB rows (TB rows for the one-pass kernel)
+  CUtensorMap tdo[kMaxRanks];   // box 64 cols x SB rows (TB rows for the one-pass kernel)
   CUtensorMap tk[kMaxRanks];    // box 64 cols x TB rows
   CUtensorMap tv[kMaxRanks];    // box 64 cols x TB rows
   RankPtrsMut dk, dv;
@@ -892,6 +892,9 @@ cudaError_t launch_common(const AttnShape& s, PrepArgs& pa, DkdvArgs& ka, DqArgs
   qa.num_m_tiles = (s.N + TB - 1) / TB;
   if (attn_bwd_onepass(s.d, deterministic) && attn_bwd_onepass_usable()) {
     ka.dqacc = Dv + static_cast<size_t>(s.P) * s.Hl * Npad;   // 512-byte aligned: Npad is a multiple of 128
+    // the one-pass kernel streams 128-row Q and dO blocks: the dQ kernel's maps
+    memcpy(ka.tq, qa.tq, sizeof(ka.tq));
+    memcpy(ka.tdo, qa.tdo, sizeof(ka.tdo));
     return launch_onepass(s, pa, ka, qa.dq, stream);
   }
   return s.d == 64 ? launch_all<64>(s, pa, ka, qa, stream) : launch_all<128>(s, pa, ka, qa, stream);
