@@ -795,7 +795,7 @@ cudaError_t launch_onepass(const AttnShape& s, const PrepArgs& pa, const DkdvArg
     cudaError_t e = cudaFuncSetAttribute(onepass::attn_bwd_onepass_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, onepass::Layout::kAlloc);
     if (e != cudaSuccess) return e;
-    dim3 grid(s.Hkvl * nranks, (s.N + TB - 1) / TB);
+    dim3 grid((s.N + TB - 1) / TB, s.Hkvl * nranks);
     onepass::attn_bwd_onepass_kernel<<<grid, onepass::kOpThreads, onepass::Layout::kAlloc, stream>>>(ka);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
