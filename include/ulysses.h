@@ -363,6 +363,64 @@ ULY_API int ulysses_attn_bwd_onepass_layout_fits(uint32_t dyn_smem_offset);
  * ulysses_get_device_status(). Use ulysses_set_wait_limit() first to keep it short. */
 ULY_API uly_status ulysses_selftest_bounded_wait(cudaStream_t stream);
 
+/* ---------------------------------------------------------------- host-to-host steps
+ * The layer with its inputs and outputs in HOST memory (theaicatchup.com, "How
+ * Does Ulysses Sequence Parallelism Actually Work?": sequence shards in,
+ * sequence shards out). Each submitted step copies the step's sequence shards
+ * Q, K, V (and dO when backward != 0) from host memory to the GPU, runs
+ * ulysses_a2a_seq_to_head, ulysses_attn_fwd, ulysses_a2a_head_to_seq of O (and
+ * ulysses_a2a_seq_to_head of dO, ulysses_attn_bwd, ulysses_a2a_head_to_seq of
+ * dQ, dK, dV), and copies O (and dQ, dK, dV) back to host memory. Results are
+ * bit-identical to those calls made one by one.
+ *
+ * Copies in, compute and copies out run on three streams the handle creates,
+ * with two alternating sets of sequence-side device buffers, so the copies of
+ * neighbouring steps overlap this step's kernels and PCIe carries both
+ * directions at once. The caller owns the device memory: one scratch buffer
+ * of ulysses_host_pipeline_scratch_bytes() bytes, 256-byte aligned, that must
+ * outlive the handle and is used by nothing else meanwhile. The handle owns
+ * only host memory, its streams and its events. */
+typedef struct uly_host_pipeline uly_host_pipeline;
+
+/* Scratch bytes for the shape (0 if the shape is unsupported). Two sets of
+ * sequence-side buffers, the head-side buffers, the LSE and, with backward,
+ * the ulysses_attn_bwd workspace of the given mode. */
+ULY_API size_t ulysses_host_pipeline_scratch_bytes(int64_t N, int P, int H, int H_kv, int d, int backward,
+                                                   int deterministic);
+
+/* Creates a handle over `scratch` (device, 256-byte aligned, scratch_bytes at
+ * least the size above). *out is NULL on failure. Status: ULY_ERR_INVALID_ARG
+ * (NULL out or scratch, misaligned or short scratch), ULY_ERR_UNSUPPORTED
+ * (shape), ULY_ERR_CUDA (stream or event creation). */
+ULY_API uly_status ulysses_host_pipeline_create(int64_t N, int P, int H, int H_kv, int d, int backward,
+                                                int deterministic, void* scratch, size_t scratch_bytes,
+                                                uly_host_pipeline** out);
+
+/* Enqueues one step and returns without waiting. *_host: HOST arrays of P
+ * HOST pointers, one sequence shard each ([N/P, Hx, d] bf16, 16-byte aligned;
+ * pinned memory for the copies to be asynchronous). dO, dQ, dK, dV are read
+ * only with backward (may be NULL otherwise). The input shards must stay
+ * unchanged and the output shards unread until the step's copies are done:
+ * after `after` (if not NULL) has completed, or after
+ * ulysses_host_pipeline_synchronize(). cu_seqlens as everywhere (DEVICE
+ * array, or NULL); softmax_scale 0 = 1/sqrt(d). before / after: caller-owned
+ * CUDA events (or NULL) recorded on the copy-in stream before the step's first
+ * copy and on the copy-out stream after its last. Validation failures return
+ * before anything is enqueued; a launch failure returns ULY_ERR_CUDA. */
+ULY_API uly_status ulysses_host_pipeline_submit(uly_host_pipeline* pipe, const void* const* q_host,
+                                                const void* const* k_host, const void* const* v_host,
+                                                const void* const* do_host, void* const* o_host,
+                                                void* const* dq_host, void* const* dk_host, void* const* dv_host,
+                                                const int32_t* cu_seqlens, int num_seqs, float softmax_scale,
+                                                cudaEvent_t before, cudaEvent_t after);
+
+/* Waits for every step submitted so far. */
+ULY_API uly_status ulysses_host_pipeline_synchronize(uly_host_pipeline* pipe);
+
+/* Waits for the submitted steps, then releases the handle's streams, events
+ * and host memory (not the scratch buffer). NULL is accepted. */
+ULY_API uly_status ulysses_host_pipeline_destroy(uly_host_pipeline* pipe);
+
 #ifdef __cplusplus
 }
 #endif

@@ -203,3 +203,38 @@ def test_onepass_backward_selection_rule(L):
     # the fitting offsets are those within a fixed distance below each boundary
     pads = sorted({(1024 - o % 1024) % 1024 for o in fits})
     assert pads == list(range(0, pads[-1] + 1, 16)) and pads[-1] < 1024
+
+
+def test_host_pipeline_scratch_size_and_validation(L):
+    """The host-to-host pipeline's scratch size is the sum of its parts (two
+    sets of sequence-side shards, the head-side shards, the LSE and the
+    backward workspace, each rounded up to 256 bytes), unsupported shapes give
+    0, and create/submit reject bad arguments before touching CUDA."""
+    import ctypes
+    N, P, H, H_kv, d = 1024, 4, 8, 4, 128
+    rnd = lambda x: (x + 255) // 256 * 256
+    q = N // P * H * d * 2
+    kv = N // P * H_kv * d * 2
+    lse = H // P * N * 4
+    for bwd, det in ((0, 0), (1, 0), (1, 1)):
+        ins = [q, kv, kv] + ([q] if bwd else [])
+        outs = [q] + ([q, kv, kv] if bwd else [])
+        heads = [q, kv, kv, q] + ([q, q, kv, kv] if bwd else [])
+        want = 2 * P * sum(rnd(x) for x in ins + outs) + P * sum(rnd(x) for x in heads) + P * rnd(lse)
+        if bwd:
+            want += rnd(L.ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, det))
+        assert L.ulysses_host_pipeline_scratch_bytes(N, P, H, H_kv, d, bwd, det) == want, (bwd, det)
+    assert L.ulysses_host_pipeline_scratch_bytes(N, P, H, H_kv, 96, 1, 0) == 0
+    assert L.ulysses_host_pipeline_scratch_bytes(N + 1, P, H, H_kv, d, 1, 0) == 0
+    h = ctypes.c_void_p()
+    n = L.ulysses_host_pipeline_scratch_bytes(N, P, H, H_kv, d, 1, 0)
+    assert L.ulysses_host_pipeline_create(N, P, H, H_kv, d, 1, 0, None, n, ctypes.byref(h)) == 1
+    assert L.ulysses_host_pipeline_create(N, P, H, H_kv, d, 1, 0, 1 << 40, n - 1, ctypes.byref(h)) == 1
+    assert L.ulysses_host_pipeline_create(N, P, H, H_kv, d, 1, 0, (1 << 40) + 16, n, ctypes.byref(h)) == 1
+    assert L.ulysses_host_pipeline_create(N, P, H, H_kv, 96, 1, 0, 1 << 40, n, ctypes.byref(h)) == 2
+    assert L.ulysses_host_pipeline_create(N, P, H, H_kv, d, 1, 0, 1 << 40, n, None) == 1
+    assert not h.value
+    assert L.ulysses_host_pipeline_submit(None, None, None, None, None, None, None, None, None, None, 0, 0.0,
+                                          None, None) == 1
+    assert L.ulysses_host_pipeline_synchronize(None) == 1
+    assert L.ulysses_host_pipeline_destroy(None) == 0

@@ -1,8 +1,11 @@
-"""HostPipeline (inputs and results in pinned host memory, copies of
-neighbouring steps overlapping the kernels on separate streams) against the
-plain device-resident layer: several different steps submitted back to back
-must each give exactly the results of running that step alone, which catches
-a step reading or overwriting the other buffer set too early."""
+"""The C-ABI host pipeline (ulysses_host_pipeline_*, through HostPipeline:
+inputs and results in pinned host memory, copies of neighbouring steps
+overlapping the kernels on the library's three streams) against the plain
+device-resident layer: several different steps submitted back to back must
+each give exactly the results of running that step alone, which catches a
+step reading or overwriting the other buffer set too early. With the
+one-pass backward, dQ is summed by fp32 reductions in a timing-dependent
+order, so it is compared to one bf16 step; everything else bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -18,12 +21,12 @@ def _host_shards(a, P):
             for p in range(P)]
 
 
-@pytest.mark.parametrize("backward", [True, False])
-def test_pipelined_steps_equal_single_steps(backward):
+@pytest.mark.parametrize("backward,deterministic", [(True, True), (False, True), (True, False)])
+def test_pipelined_steps_equal_single_steps(backward, deterministic):
     import ulysses_sequence_parallelism_b200 as U
     N, P, H, H_kv, d = 1024, 4, 8, 4, 128
     cu = torch.tensor([0, 300, 301, 1024], dtype=torch.int32, device="cuda")
-    layer = U.UlyssesLayer(N, P, H, H_kv, d, cu_seqlens=cu, backward=backward, deterministic=True)
+    layer = U.UlyssesLayer(N, P, H, H_kv, d, cu_seqlens=cu, backward=backward, deterministic=deterministic)
     steps = []
     for seed in range(5):
         rng = np.random.Generator(np.random.PCG64(100 + seed))
@@ -54,4 +57,10 @@ def test_pipelined_steps_equal_single_steps(backward):
         torch.cuda.synchronize()
         for name, ts in ref.items():
             for r, (a, b) in enumerate(zip(got[name], ts)):
-                assert torch.equal(a.view(torch.int16), b.cpu().view(torch.int16)), (name, r)
+                if name == "dq" and not deterministic:
+                    bf = b.cpu().float()
+                    step = torch.clamp(bf.abs(), min=2.0 ** -126) * 2.0 ** -7   # one bf16 step (upper bound)
+                    assert ((a.float() - bf).abs() <= step).all(), (name, r)
+                else:
+                    assert torch.equal(a.view(torch.int16), b.cpu().view(torch.int16)), (name, r)
+    hp.close()

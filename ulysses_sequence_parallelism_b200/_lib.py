@@ -56,9 +56,15 @@ _SIGS = {
                              _i, ctypes.c_float, _i, _v, ctypes.c_size_t, _i, _i, _v],
     "ulysses_attn_bwd_noalloc": [_vpp, _vpp, _vpp, _vpp, _fpp, _vpp, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _v, _i,
                                  _i, ctypes.c_float, _i, _i, _v],
+    "ulysses_host_pipeline_scratch_bytes": [_i64, _i, _i, _i, _i, _i, _i],
+    "ulysses_host_pipeline_create": [_i64, _i, _i, _i, _i, _i, _i, _v, ctypes.c_size_t, ctypes.POINTER(_v)],
+    "ulysses_host_pipeline_submit": [_v, _vpp, _vpp, _vpp, _vpp, _vpp, _vpp, _vpp, _vpp, _v, _i, ctypes.c_float,
+                                     _v, _v],
+    "ulysses_host_pipeline_synchronize": [_v],
+    "ulysses_host_pipeline_destroy": [_v],
 }
 _RES = {"ulysses_attn_bwd_workspace_size": ctypes.c_size_t, "ulysses_status_string": ctypes.c_char_p,
-        "ulysses_set_wait_limit": None}
+        "ulysses_set_wait_limit": None, "ulysses_host_pipeline_scratch_bytes": ctypes.c_size_t}
 
 
 def lib():

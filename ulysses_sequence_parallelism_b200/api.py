@@ -406,75 +406,88 @@ class UlyssesLayer:
 
 
 class HostPipeline:
-    """Layer steps whose inputs and results live in pinned host memory.
+    """Layer steps whose inputs and results live in host memory, through the
+    C-ABI host pipeline (``ulysses_host_pipeline_*``; this class only
+    marshals arguments and owns the device scratch buffer).
 
-    ``submit(host_in, host_out)`` enqueues one training step of ``layer``
-    (forward + backward when the layer has backward buffers): the host->device
-    copy of the step's sequence shards (Q, K, V, dO), the layer's kernels, and
-    the device->host copy of its results (O, dQ, dK, dV). Copies in, compute
-    and copies out run on three streams with two device buffer sets, so the
-    copies of neighbouring steps overlap this step's kernels and PCIe moves
-    data in both directions at once. Results of a step are in ``host_out``
-    once ``synchronize()`` returns (or its ``done`` event has completed).
+    ``submit(host_in, host_out)`` enqueues one step of ``layer``'s shape and
+    options (forward + backward when the layer has backward buffers): the
+    host->device copies of the step's sequence shards (Q, K, V, dO), the
+    layer's kernels, and the device->host copies of its results (O, dQ, dK,
+    dV). Copies in, compute and copies out run on three streams of the library
+    with two device buffer sets, so the copies of neighbouring steps overlap
+    this step's kernels and PCIe carries both directions at once. Results of a
+    step are in ``host_out`` once ``synchronize()`` returns (or once the
+    ``after`` event given to ``submit`` has completed).
 
     host_in:  {"q": [P tensors], "k": [...], "v": [...], "do": [...]}
     host_out: {"o": [...], "dq": [...], "dk": [...], "dv": [...]}
-    (pinned CPU tensors shaped like the sequence shards; "do", "dq", "dk",
-    "dv" only with backward).
+    (pinned CPU bf16 tensors shaped like the sequence shards; "do", "dq",
+    "dk", "dv" only with backward). The layer's own device buffers are not
+    used: the pipeline has its own in its scratch buffer.
     """
 
     def __init__(self, layer: "UlyssesLayer", device="cuda"):
         self.layer = layer
+        self.bwd = bool(layer.backward_enabled)
         N, P, H, H_kv, d = layer.N, layer.P, layer.H, layer.H_kv, layer.d
-        bf = torch.bfloat16
-        n = N // P
-        shard = lambda hx: [torch.empty(n, hx, d, dtype=bf, device=device) for _ in range(P)]
-        self.bwd = layer.backward_enabled
-        self.ins = [{"q": shard(H), "k": shard(H_kv), "v": shard(H_kv), **({"do": shard(H)} if self.bwd else {})}
-                    for _ in range(2)]
-        self.outs = [{"o": shard(H), **({"dq": shard(H), "dk": shard(H_kv), "dv": shard(H_kv)} if self.bwd else {})}
-                     for _ in range(2)]
-        self.s_in = torch.cuda.Stream(device=device)
-        self.s_comp = torch.cuda.Stream(device=device)
-        self.s_out = torch.cuda.Stream(device=device)
-        self.in_free = [None, None]      # compute finished reading input set j
-        self.out_free = [None, None]     # copy-out finished reading output set j
-        self.k = 0
+        det = int(bool(layer.deterministic))
+        nbytes = int(lib().ulysses_host_pipeline_scratch_bytes(N, P, H, H_kv, d, int(self.bwd), det))
+        if nbytes == 0:
+            raise UlyssesError("ulysses_host_pipeline_scratch_bytes", 2)
+        self.scratch = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        handle = ctypes.c_void_p()
+        check("ulysses_host_pipeline_create",
+              lib().ulysses_host_pipeline_create(N, P, H, H_kv, d, int(self.bwd), det,
+                                                 ctypes.c_void_p(self.scratch.data_ptr()), nbytes,
+                                                 ctypes.byref(handle)))
+        self.handle = handle
+        self._cu, self._ns = _cu(layer.cu)
 
-    def submit(self, host_in, host_out):
-        j = self.k & 1
-        self.k += 1
-        dev_in, dev_out = self.ins[j], self.outs[j]
-        loaded = torch.cuda.Event()
-        with torch.cuda.stream(self.s_in):
-            if self.in_free[j] is not None:
-                self.s_in.wait_event(self.in_free[j])
-            for name, bufs in dev_in.items():
-                for dst, src in zip(bufs, host_in[name]):
-                    dst.copy_(src, non_blocking=True)
-            loaded.record(self.s_in)
-        computed, in_free = torch.cuda.Event(), torch.cuda.Event()
-        with torch.cuda.stream(self.s_comp):
-            self.s_comp.wait_event(loaded)
-            if self.out_free[j] is not None:
-                self.s_comp.wait_event(self.out_free[j])
-            L = self.layer
-            L.forward(dev_in["q"], dev_in["k"], dev_in["v"], dev_out["o"])
-            if self.bwd:
-                L.backward(dev_in["do"], dev_out["dq"], dev_out["dk"], dev_out["dv"])
-            in_free.record(self.s_comp)
-            computed.record(self.s_comp)
-        self.in_free[j] = in_free
-        done = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(self.s_out):
-            self.s_out.wait_event(computed)
-            for name, bufs in dev_out.items():
-                for dst, src in zip(host_out[name], bufs):
-                    dst.copy_(src, non_blocking=True)
-            done.record(self.s_out)
-        self.out_free[j] = done
-        return done
+    @staticmethod
+    def _host_ptrs(ts, P):
+        if ts is None:
+            return None
+        if len(ts) != P:
+            raise ValueError(f"expected {P} host shards, got {len(ts)}")
+        arr = (ctypes.c_void_p * P)()
+        for r, t in enumerate(ts):
+            if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+                raise ValueError(f"rank {r}: need a contiguous host bf16 tensor")
+            arr[r] = t.data_ptr()
+        return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+
+    @staticmethod
+    def _event(ev):
+        if ev is None:
+            return None
+        if ev.cuda_event == 0:          # torch creates the event at its first record
+            ev.record()
+        return ctypes.c_void_p(ev.cuda_event)
+
+    def submit(self, host_in, host_out, before=None, after=None):
+        """before / after: optional torch.cuda.Event, recorded on the copy-in
+        stream before the step's first copy and on the copy-out stream after
+        its last."""
+        P = self.layer.P
+        used = ("q", "k", "v", "o") + (("do", "dq", "dk", "dv") if self.bwd else ())
+        hp = lambda dct, key: self._host_ptrs(dct.get(key), P) if key in used else None
+        check("ulysses_host_pipeline_submit",
+              lib().ulysses_host_pipeline_submit(self.handle, hp(host_in, "q"), hp(host_in, "k"), hp(host_in, "v"),
+                                                 hp(host_in, "do"), hp(host_out, "o"), hp(host_out, "dq"),
+                                                 hp(host_out, "dk"), hp(host_out, "dv"), self._cu, self._ns,
+                                                 float(self.layer.scale), self._event(before), self._event(after)))
 
     def synchronize(self):
-        for s in (self.s_in, self.s_comp, self.s_out):
-            s.synchronize()
+        check("ulysses_host_pipeline_synchronize", lib().ulysses_host_pipeline_synchronize(self.handle))
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            lib().ulysses_host_pipeline_destroy(self.handle)
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -8,3 +8,4 @@
 #include "proj_sm100.cu"
 #include "api.cu"
 #include "bwd_noalloc.cu"
+#include "host_pipeline.cu"
