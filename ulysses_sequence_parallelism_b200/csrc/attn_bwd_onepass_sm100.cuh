@@ -123,14 +123,16 @@ __global__ void __launch_bounds__(kOpThreads, 1) attn_bwd_onepass_kernel(const _
   volatile uint32_t* slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // blockIdx.x is the key block: the CTAs resident together belong to one
-  // (rank, kv head) and stream the same Q/dO blocks into the same
-  // accumulator rows, which then stay in L2 (DRAM traffic 3.8 GB per call at
-  // varlen 64K, against 8.5 GB with the kv head as the fast index).
-  const int g = blockIdx.y % a.Hkvl;
-  const int r = a.rank_lo + blockIdx.y / a.Hkvl;
+  // kb_fast: blockIdx.x is the key block, so the CTAs resident together
+  // belong to one (rank, kv head) and stream the same Q/dO blocks into the
+  // same accumulator rows, which then stay in L2. Else blockIdx.x is the
+  // (rank, kv head) and every pair's heaviest key blocks launch first (the
+  // host picks; see launch_onepass).
+  const int combo = a.kb_fast ? blockIdx.y : blockIdx.x;
+  const int g = combo % a.Hkvl;
+  const int r = a.rank_lo + combo / a.Hkvl;
   const int N = a.N;
-  const int n0 = blockIdx.x * TB;
+  const int n0 = (a.kb_fast ? blockIdx.x : blockIdx.y) * TB;
   const int n_last = min(n0 + TB, N) - 1;
   const int doc_end_first = doc_end_of(a.cu, a.num_seqs, n0, N);
   const int m_end = doc_end_of(a.cu, a.num_seqs, n_last, N);
