@@ -108,6 +108,26 @@ def test_onepass_and_twopass_backward_agree():
     assert np.all(np.abs(again["dq"] - one["dq"]) <= ulp)
 
 
+@pytest.mark.parametrize("N,P,cu", [
+    (296 * 128 + 77, 1, [0, 5000, 5001, 20000, 296 * 128 + 77]),   # 297 key blocks, ragged last block
+    (2 * 148 * 128, 2, None),                                         # exactly the two-wave threshold
+])
+def test_onepass_key_block_first_launch_agrees_with_two_pass(N, P, cu):
+    """From two waves of key blocks (296 on 148 SMs) the one-pass kernel runs
+    with the key block as the grid's fast index; the small cases above run the
+    other order. Here that path, with a ragged last key block and documents
+    straddling key blocks, against the two-pass backward: dK and dV bit for
+    bit, dQ to one bf16 step (the fp32 sums' order)."""
+    H, H_kv, d = 4, 2, 128
+    q, k, v, do = _draw(N, H, H_kv, d, seed=123)
+    two = run_gpu_layer(q, k, v, do, P, cu, deterministic=True)
+    one = run_gpu_layer(q, k, v, do, P, cu, deterministic=False)
+    for n in ("o", "dk", "dv"):
+        assert np.array_equal(one[n], two[n]), n
+    ulp = np.abs(two["dq"]) * 2.0 ** -7 + 1e-5 * np.abs(two["dq"]).max()
+    assert np.all(np.abs(one["dq"] - two["dq"]) <= ulp)
+
+
 def test_softmax_scale_argument():
     """An explicit softmax_scale (0.09, not the default 1/sqrt(64) = 0.125) is
     honoured by forward and backward."""
