@@ -24,7 +24,8 @@
  *     library never allocates or frees device memory.
  *   - Every device pointer must be 16-byte aligned.
  *   - Calls are asynchronous on `stream` (0 = legacy default stream) and do
- *     not synchronise, except ulysses_get_device_status().
+ *     not synchronise, except ulysses_get_device_status() and the host
+ *     pipeline's synchronize/destroy (which run on the handle's own streams).
  *   - Arguments are validated before any launch. On ULY_ERR_INVALID_ARG or
  *     ULY_ERR_UNSUPPORTED nothing is launched and no memory is touched. A
  *     launch failure returns ULY_ERR_CUDA. Nothing aborts or traps.
