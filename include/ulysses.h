@@ -380,7 +380,9 @@ ULY_API uly_status ulysses_selftest_bounded_wait(cudaStream_t stream);
  * directions at once. The caller owns the device memory: one scratch buffer
  * of ulysses_host_pipeline_scratch_bytes() bytes, 256-byte aligned, that must
  * outlive the handle and is used by nothing else meanwhile. The handle owns
- * only host memory, its streams and its events. */
+ * only host memory, its streams and its events. A handle is not thread-safe:
+ * calls on one handle must not overlap (different handles may be used from
+ * different threads). */
 typedef struct uly_host_pipeline uly_host_pipeline;
 
 /* Scratch bytes for the shape (0 if the shape is unsupported). Two sets of
