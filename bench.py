@@ -605,9 +605,12 @@ def main():
         f_fwd_ms = sum(e[0].elapsed_time(e[1]) for e in fev) / args.steps
         f_bwd_ms = sum(e[1].elapsed_time(e[2]) for e in fev) / args.steps
         f_ms, f_val = aggregate_over_ranks(f_fwd_ms + f_bwd_ms, N, world, reduce_max)
+        staged = (not args.deterministic) and d == 128   # one-pass: Q and dO staged in head shards
         fused = {"value": f_val, "unit": "tokens/s", "ms_per_step": f_ms, "attn_fwd_seq_ms": f_fwd_ms,
-                 "attn_bwd_seq_ms": f_bwd_ms, "gpu_launches_per_step": 1 + 3,
-                 "note": "all-to-alls folded into the attention kernels' addressing (no permute launches)"}
+                 "attn_bwd_seq_ms": f_bwd_ms, "gpu_launches_per_step": 1 + 3 + (2 if staged else 0),
+                 "note": "all-to-alls folded into the attention kernels' addressing; the one-pass backward "
+                         "first copies Q and dO into head shards in its workspace (2 permute launches), "
+                         "O, dQ, dK, dV go straight to the sequence shards"}
         del lf
 
     # ---------------------------------------------------------------- head fragmentation (NEXT-3)

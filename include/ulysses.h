@@ -294,9 +294,20 @@ ULY_API uly_status ulysses_attn_bwd(
  * the head->seq all-to-all of dQ, dK, dV, reading Q, K, V, O, dO from the
  * sequence shards and writing dQ, dK, dV into them (all arrays: P sequence
  * shards; lse_head: per rank in range, from ulysses_attn_fwd_seq or
- * ulysses_attn_fwd). Workspace and `deterministic` as ulysses_attn_bwd;
- * bit-identical to the separate calls (for dQ with deterministic == 0: up to
- * the run-to-run order of the fp32 sums). Needs (N/P) % 128 == 0; otherwise ULY_ERR_UNSUPPORTED. */
+ * ulysses_attn_fwd). Workspace and `deterministic` as ulysses_attn_bwd (at
+ * least ulysses_attn_bwd_workspace_size() bytes); given
+ * ulysses_attn_bwd_seq_workspace_size() bytes, the one-pass mode first copies
+ * Q and dO into head shards inside the workspace (two permute launches) and
+ * streams them from there, which is faster than from the sequence shards.
+ * Bit-identical to the separate calls either way (for dQ with
+ * deterministic == 0: up to the run-to-run order of the fp32 sums). Needs
+ * (N/P) % 128 == 0; otherwise ULY_ERR_UNSUPPORTED. */
+/* Workspace bytes with which ulysses_attn_bwd_seq stages Q and dO in head
+ * shards: ulysses_attn_bwd_workspace_size() plus, in the one-pass mode
+ * (deterministic == 0, d == 128), 2 * P * N * (H/P) * d * 2 bytes. 0 if the
+ * shape is unsupported. */
+ULY_API size_t ulysses_attn_bwd_seq_workspace_size(int64_t N, int P, int H, int H_kv, int d, int deterministic);
+
 ULY_API uly_status ulysses_attn_bwd_seq(
     const void* const* q_seq, const void* const* k_seq, const void* const* v_seq,
     const void* const* o_seq, const float* const* lse_head, const void* const* do_seq,

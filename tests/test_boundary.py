@@ -238,3 +238,16 @@ def test_host_pipeline_scratch_size_and_validation(L):
                                           None, None) == 1
     assert L.ulysses_host_pipeline_synchronize(None) == 1
     assert L.ulysses_host_pipeline_destroy(None) == 0
+
+
+def test_seq_backward_workspace_size(L):
+    """The sequence-layout backward's larger workspace (room to stage Q and dO
+    in head shards) exists only for the one-pass mode: 2 * P * N * (H/P) * d
+    bf16 more than the plain backward's; otherwise the two sizes agree."""
+    N, P, H, H_kv = 8192, 4, 32, 8
+    for d, det in ((128, 0), (128, 1), (64, 0)):
+        base = L.ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, det)
+        seq = L.ulysses_attn_bwd_seq_workspace_size(N, P, H, H_kv, d, det)
+        extra = 2 * P * N * (H // P) * d * 2 if (d == 128 and det == 0) else 0
+        assert base > 0 and seq == base + extra, (d, det)
+    assert L.ulysses_attn_bwd_seq_workspace_size(N, P, H, H_kv, 96, 0) == 0

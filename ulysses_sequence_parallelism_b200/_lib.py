@@ -43,6 +43,7 @@ _SIGS = {
     "ulysses_attn_fwd": [_vpp, _vpp, _vpp, _vpp, _fpp, _i64, _i, _i, _i, _i, _v, _i, _i, ctypes.c_float, _i,
                          _i, _i, _v],
     "ulysses_attn_bwd_workspace_size": [_i64, _i, _i, _i, _i, _i],
+    "ulysses_attn_bwd_seq_workspace_size": [_i64, _i, _i, _i, _i, _i],
     "ulysses_attn_bwd": [_vpp, _vpp, _vpp, _vpp, _fpp, _vpp, _vpp, _vpp, _vpp, _i64, _i, _i, _i, _i, _v, _i, _i,
                          ctypes.c_float, _i, _v, ctypes.c_size_t, _i, _i, _v],
     "ulysses_status_string": [_i],
@@ -63,7 +64,7 @@ _SIGS = {
     "ulysses_host_pipeline_synchronize": [_v],
     "ulysses_host_pipeline_destroy": [_v],
 }
-_RES = {"ulysses_attn_bwd_workspace_size": ctypes.c_size_t, "ulysses_status_string": ctypes.c_char_p,
+_RES = {"ulysses_attn_bwd_workspace_size": ctypes.c_size_t, "ulysses_attn_bwd_seq_workspace_size": ctypes.c_size_t, "ulysses_status_string": ctypes.c_char_p,
         "ulysses_set_wait_limit": None, "ulysses_host_pipeline_scratch_bytes": ctypes.c_size_t}
 
 

@@ -19,7 +19,8 @@ from ._lib import lib, check, UlyssesError, MAX_RANKS
 
 __all__ = [
     "ulysses_a2a_seq_to_head", "ulysses_a2a_head_to_seq", "ulysses_attn_fwd", "ulysses_attn_bwd",
-    "ulysses_attn_bwd_workspace_size", "ulysses_get_device_status", "ulysses_set_wait_limit",
+    "ulysses_attn_bwd_workspace_size", "ulysses_attn_bwd_seq_workspace_size", "ulysses_get_device_status",
+    "ulysses_set_wait_limit",
     "ulysses_selftest_bounded_wait", "ulysses_attn_fwd_seq", "ulysses_attn_bwd_seq", "UlyssesLayer",
     "HostPipeline", "ulysses_a2a_seq_to_head_frag", "ulysses_a2a_head_to_seq_frag",
     "ulysses_qkv_proj_seq_to_head", "ulysses_out_proj_head_to_seq", "ulysses_out_proj_bwd",
@@ -193,6 +194,10 @@ def ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, deterministic=False) -> in
     return int(lib().ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, int(bool(deterministic))))
 
 
+def ulysses_attn_bwd_seq_workspace_size(N, P, H, H_kv, d, deterministic=False) -> int:
+    return int(lib().ulysses_attn_bwd_seq_workspace_size(N, P, H, H_kv, d, int(bool(deterministic))))
+
+
 def ulysses_attn_bwd(q_head, k_head, v_head, o_head, lse_head, do_head, dq_head, dk_head, dv_head, N, P, H,
                      H_kv, d, workspace: torch.Tensor, cu_seqlens=None, max_seqlen=0, softmax_scale=0.0,
                      rank_lo=0, rank_hi=None, stream=None, deterministic=False):
@@ -282,7 +287,9 @@ class UlyssesLayer:
                 self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
         elif self.backward_enabled:
             self.do_h, self.dq_h, self.dk_h, self.dv_h = mk(H), mk(H), mk(H_kv), mk(H_kv)
-            ws = ulysses_attn_bwd_workspace_size(N, P, H, H_kv, d, deterministic)
+            # fused: room for the backward to stage Q and dO in head shards
+            size = ulysses_attn_bwd_seq_workspace_size if fused else ulysses_attn_bwd_workspace_size
+            ws = size(N, P, H, H_kv, d, deterministic)
             self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
 
     def forward_projected(self, x_seq: List[torch.Tensor], w_qkv: torch.Tensor, w_o: torch.Tensor,

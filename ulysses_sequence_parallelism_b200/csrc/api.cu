@@ -404,7 +404,12 @@ uly_status ulysses_attn_bwd_seq(const void* const* q_seq, const void* const* k_s
   uly::AttnShape s{static_cast<int>(N), P, H / P, H_kv / P, d, cu_seqlens, cu_seqlens ? num_seqs : 1,
                    resolve_scale(softmax_scale, d), rank_lo, rank_hi};
   return from_cuda(uly::launch_attn_bwd_seq(s, q_seq, k_seq, v_seq, o_seq, lse_head, do_seq, dq_seq, dk_seq,
-                                            dv_seq, workspace, deterministic, stream));
+                                            dv_seq, workspace, workspace_bytes, deterministic, stream));
+}
+
+size_t ulysses_attn_bwd_seq_workspace_size(int64_t N, int P, int H, int H_kv, int d, int deterministic) {
+  if (check_shape(N, P, H, H_kv, d, 0, P > 0 ? P : 1) != ULY_OK) return 0;
+  return uly::attn_bwd_seq_workspace_bytes(N, P, H / P, d, deterministic);
 }
 
 const char* ulysses_status_string(uly_status s) {

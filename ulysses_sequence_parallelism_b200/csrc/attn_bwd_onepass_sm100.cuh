@@ -163,8 +163,12 @@ __global__ void __launch_bounds__(kOpThreads, 1) attn_bwd_onepass_kernel(const _
     {
       auto shard_of = [&](int tok) { return a.seq ? tok / a.n_loc : r; };
       auto row_in = [&](int tok) { return a.seq ? tok - (tok / a.n_loc) * a.n_loc : tok; };
-      const int qx0 = a.seq ? r * a.Hl * D : 0, kx0 = a.seq ? (r * a.Hkvl + g) * D : g * D;
-      if (!a.seq && lane == 0) {
+      // Q and dO: sequence shards (qdo_seq) or head shards (also in the
+      // sequence-layout call, which may stage them there first)
+      auto q_shard = [&](int tok) { return a.qdo_seq ? tok / a.n_loc : r; };
+      auto q_row = [&](int tok) { return a.qdo_seq ? tok - (tok / a.n_loc) * a.n_loc : tok; };
+      const int qx0 = a.qdo_seq ? r * a.Hl * D : 0, kx0 = a.seq ? (r * a.Hkvl + g) * D : g * D;
+      if (!a.qdo_seq && lane == 0) {
         tma_prefetch_desc(&a.tq[r]);
         tma_prefetch_desc(&a.tdo[r]);
       }
@@ -185,9 +189,9 @@ __global__ void __launch_bounds__(kOpThreads, 1) attn_bwd_onepass_kernel(const _
         mbar_arrive_expect_tx_w(st_full(s), 2 * L::kBlk + L::kVecStage);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf) {
-          tma_load_2d_w(stg + hf * L::kHalf, &a.tq[shard_of(m0)], st_full(s), qx0 + h * D + hf * 64, row_in(m0));
-          tma_load_2d_w(stg + L::kBlk + hf * L::kHalf, &a.tdo[shard_of(m0)], st_full(s), qx0 + h * D + hf * 64,
-                        row_in(m0));
+          tma_load_2d_w(stg + hf * L::kHalf, &a.tq[q_shard(m0)], st_full(s), qx0 + h * D + hf * 64, q_row(m0));
+          tma_load_2d_w(stg + L::kBlk + hf * L::kHalf, &a.tdo[q_shard(m0)], st_full(s), qx0 + h * D + hf * 64,
+                        q_row(m0));
         }
         const int64_t vo = (static_cast<int64_t>(r) * a.Hl + h) * a.Npad + m0;
         bulk_load_w(sbase + L::kVec + s * L::kVecStage, a.lse2 + vo, QB * 4, st_full(s));

@@ -135,6 +135,7 @@ struct DkdvArgs {
   int rank_lo;
   int seq, n_loc, P;
   int kb_fast;                  // one-pass kernel only: blockIdx.x is the key block (else the kv head)
+  int qdo_seq;                  // one-pass kernel only: tq/tdo map sequence shards (else head shards)
 };
 
 template <int D>
@@ -855,6 +856,12 @@ bool attn_bwd_onepass_usable() {
   return cache[dev] == 1;
 }
 
+size_t attn_bwd_seq_workspace_bytes(int64_t N, int P, int Hl, int d, int deterministic) {
+  size_t bytes = attn_bwd_workspace_bytes(N, P, Hl, d, deterministic);
+  if (attn_bwd_onepass(d, deterministic)) bytes += 2 * static_cast<size_t>(P) * N * Hl * d * 2;
+  return bytes;
+}
+
 size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d, int deterministic) {
   const int64_t npad = (N + bwd_sm100::TB - 1) / bwd_sm100::TB * bwd_sm100::TB;
   size_t bytes = 2 * static_cast<size_t>(P) * Hl * npad * sizeof(float);
@@ -878,8 +885,10 @@ int device_sm_count() {
 }
 
 // Fills everything but the per-buffer pointers and tensor maps, then launches.
+// qdo_head (seq == 1 only): qa.tq / qa.tdo map head-sharded copies of Q and dO
+// instead of the sequence shards.
 cudaError_t launch_common(const AttnShape& s, PrepArgs& pa, DkdvArgs& ka, DqArgs& qa, void* workspace, int seq,
-                          int deterministic, cudaStream_t stream) {
+                          int deterministic, cudaStream_t stream, bool qdo_head = false) {
   const int Npad = padded_rows(s.N);
   float* lse2 = static_cast<float*>(workspace);
   float* Dv = lse2 + static_cast<size_t>(s.P) * s.Hl * Npad;
@@ -891,6 +900,7 @@ cudaError_t launch_common(const AttnShape& s, PrepArgs& pa, DkdvArgs& ka, DqArgs
   pa.rank_lo = s.rank_lo;
   pa.nranks = s.rank_hi - s.rank_lo;
   pa.seq = ka.seq = qa.seq = seq;
+  ka.qdo_seq = seq && !qdo_head ? 1 : 0;
   pa.n_loc = ka.n_loc = qa.n_loc = s.N / s.P;
   pa.P = ka.P = qa.P = s.P;
   ka.lse2 = qa.lse2 = lse2;
@@ -961,7 +971,8 @@ cudaError_t launch_attn_bwd(const AttnShape& s, const void* const* q, const void
 cudaError_t launch_attn_bwd_seq(const AttnShape& s, const void* const* q_seq, const void* const* k_seq,
                                 const void* const* v_seq, const void* const* o_seq, const float* const* lse,
                                 const void* const* do_seq, void* const* dq_seq, void* const* dk_seq,
-                                void* const* dv_seq, void* workspace, int deterministic, cudaStream_t stream) {
+                                void* const* dv_seq, void* workspace, size_t workspace_bytes, int deterministic,
+                                cudaStream_t stream) {
   using namespace bwd_sm100;
   EncodeTiledFn enc = get_encode();
   if (enc == nullptr) return cudaErrorNotSupported;
@@ -986,7 +997,36 @@ cudaError_t launch_attn_bwd_seq(const AttnShape& s, const void* const* q_seq, co
     qa.dq.p[p] = dq_seq[p];
   }
   for (int r = s.rank_lo; r < s.rank_hi; ++r) pa.lse.p[r] = lse[r];
-  return launch_common(s, pa, ka, qa, workspace, 1, deterministic, stream);
+  // One-pass mode with room in the workspace: stage Q and dO in head shards
+  // (one permute launch each) and let the kernel stream them from there; it
+  // reads 128-row blocks whose rows are (H/P)*d*2 bytes apart instead of
+  // H*d*2 in the sequence shards, which the TMA serves faster.
+  bool qdo_head = false;
+  if (attn_bwd_onepass(s.d, deterministic) && attn_bwd_onepass_usable() &&
+      workspace_bytes >= attn_bwd_seq_workspace_bytes(s.N, s.P, s.Hl, s.d, deterministic)) {
+    const size_t shard = static_cast<size_t>(s.N) * s.Hl * s.d * 2;
+    char* base = static_cast<char*>(workspace) + attn_bwd_workspace_bytes(s.N, s.P, s.Hl, s.d, deterministic);
+    void* qh[kMaxRanks] = {};
+    void* doh[kMaxRanks] = {};
+    for (int r = s.rank_lo; r < s.rank_hi; ++r) {
+      qh[r] = base + static_cast<size_t>(r) * shard;
+      doh[r] = base + static_cast<size_t>(s.P + r) * shard;
+    }
+    const int hx[3] = {s.Hl * s.P, s.Hkvl * s.P, s.Hkvl * s.P};
+    const void* const* src_q[3] = {q_seq, nullptr, nullptr};
+    void* const* dst_q[3] = {qh, nullptr, nullptr};
+    const void* const* src_do[3] = {do_seq, nullptr, nullptr};
+    void* const* dst_do[3] = {doh, nullptr, nullptr};
+    cudaError_t e = launch_permute(true, src_q, dst_q, hx, s.N, s.P, s.d, s.rank_lo, s.rank_hi, stream);
+    if (e == cudaSuccess) e = launch_permute(true, src_do, dst_do, hx, s.N, s.P, s.d, s.rank_lo, s.rank_hi, stream);
+    if (e != cudaSuccess) return e;
+    const int64_t qeh = static_cast<int64_t>(s.Hl) * s.d;
+    for (int r = s.rank_lo; r < s.rank_hi; ++r)
+      if (!encode(enc, &qa.tq[r], qh[r], s.N, qeh, TB) || !encode(enc, &qa.tdo[r], doh[r], s.N, qeh, TB))
+        return cudaErrorInvalidValue;
+    qdo_head = true;
+  }
+  return launch_common(s, pa, ka, qa, workspace, 1, deterministic, stream, qdo_head);
 }
 
 }  // namespace uly

@@ -44,11 +44,16 @@ cudaError_t launch_attn_fwd_seq(const AttnShape& s, const void* const* q_seq, co
 cudaError_t launch_attn_bwd_seq(const AttnShape& s, const void* const* q_seq, const void* const* k_seq,
                                 const void* const* v_seq, const void* const* o_seq, const float* const* lse,
                                 const void* const* do_seq, void* const* dq_seq, void* const* dk_seq,
-                                void* const* dv_seq, void* workspace, int deterministic, cudaStream_t stream);
+                                void* const* dv_seq, void* workspace, size_t workspace_bytes, int deterministic,
+                                cudaStream_t stream);
 
 // deterministic == 0 with d == 128 selects the one-pass backward (fp32 dQ
 // accumulator in the workspace); everything else runs the two-pass kernels.
 size_t attn_bwd_workspace_bytes(int64_t N, int P, int Hl, int d, int deterministic);
+// The sequence-layout backward's workspace: the above plus, for the one-pass
+// kernel, head-sharded copies of Q and dO (staged by a permute, since the
+// kernel streams them faster from head shards than from sequence shards).
+size_t attn_bwd_seq_workspace_bytes(int64_t N, int P, int Hl, int d, int deterministic);
 // Whether the one-pass kernel's shared-memory layout fits when its dynamic
 // shared memory starts dyn_base_offset bytes into the CTA's shared window.
 bool attn_bwd_onepass_layout_fits(uint32_t dyn_base_offset);
