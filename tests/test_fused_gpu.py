@@ -96,3 +96,42 @@ def test_fused_forward_rank_range_writes_only_its_heads():
         assert torch.all(part[p][:, :Hl] == 7.0) and torch.all(part[p][:, 3 * Hl:] == 7.0)
     for r in (1, 2):
         assert torch.equal(lse2[r], lse[r])
+
+
+@pytest.mark.parametrize("rank_lo,rank_hi", [(0, 4), (1, 3)])
+def test_seq_backward_staged_and_direct_agree(rank_lo, rank_hi):
+    """ulysses_attn_bwd_seq with the larger workspace stages Q and dO in head
+    shards first; with the plain workspace it streams them from the sequence
+    shards. Both must give the same dK, dV bits (dQ to one bf16 step: fp32
+    sums in timing order), for all ranks and for a rank range (whose heads
+    alone are written)."""
+    import ulysses_sequence_parallelism_b200 as U
+    N, P, H, H_kv, d = 1024, 4, 8, 4, 128
+    cu = torch.tensor([0, 300, 301, 777, 1024], dtype=torch.int32, device="cuda")
+    q, k, v, do = _draw(N, H, H_kv, d, seed=31)
+    qs, ks, vs, dos = (shards_to_dev(x, P) for x in (q, k, v, do))
+    o = [torch.empty(N // P, H, d, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
+    lse = [torch.empty(H // P, N, dtype=torch.float32, device="cuda") for _ in range(P)]
+    U.ulysses_attn_fwd_seq(qs, ks, vs, o, lse, N, P, H, H_kv, d, cu)
+    res = []
+    for size in (U.ulysses_attn_bwd_seq_workspace_size, U.ulysses_attn_bwd_workspace_size):
+        ws = torch.empty(size(N, P, H, H_kv, d, False), dtype=torch.uint8, device="cuda")
+        g = [[torch.full((N // P, hx, d), 3.0, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
+             for hx in (H, H_kv, H_kv)]
+        U.ulysses_attn_bwd_seq(qs, ks, vs, o, lse, dos, *g, N, P, H, H_kv, d, ws, cu,
+                               rank_lo=rank_lo, rank_hi=rank_hi)
+        torch.cuda.synchronize()
+        assert U.ulysses_get_device_status() == (0, 0)
+        res.append(g)
+    staged, direct = res
+    for t, name in enumerate(("dq", "dk", "dv")):
+        hl = (H if t == 0 else H_kv) // P
+        cols = slice(rank_lo * hl, rank_hi * hl)
+        for p in range(P):
+            a, b = staged[t][p], direct[t][p]
+            assert torch.all(a[:, :rank_lo * hl] == 3.0) and torch.all(a[:, rank_hi * hl:] == 3.0), name
+            if name == "dq":
+                fa, fb = a[:, cols].float(), b[:, cols].float()
+                assert torch.all((fa - fb).abs() <= fb.abs() * 2.0 ** -7 + 1e-5 * fb.abs().max()), name
+            else:
+                assert torch.equal(a[:, cols], b[:, cols]), name
